@@ -1,0 +1,89 @@
+"""The oracle against its pins, and the pins against planted mistakes."""
+import numpy as np
+import pytest
+
+import oracle.kv_decode as kv
+from tests import oracle_pins as pins
+
+
+@pytest.mark.parametrize("pin", pins.ALL_PINS, ids=lambda f: f.__name__)
+def test_oracle_pin(pin):
+    pin(kv)
+
+
+# --- planted mistakes: each mutation of the oracle must fail at least one pin.
+def _rope_interleaved(x, positions, base):
+    x = np.asarray(x, np.float64)
+    D = x.shape[-1]
+    ang = np.asarray(positions, np.float64)[..., None] * kv.rope_inv_freq(D, base)
+    c, s = np.cos(ang), np.sin(ang)
+    a, b = x[..., 0::2], x[..., 1::2]
+    out = np.empty_like(x)
+    out[..., 0::2] = a * c - b * s
+    out[..., 1::2] = a * s + b * c
+    return out
+
+
+def _rope_wrong_sign(x, positions, base):
+    return _orig_rope(x, -np.asarray(positions), base)
+
+
+def _inv_freq_off(head_dim, base):
+    j = np.arange(head_dim // 2, dtype=np.float64)
+    return np.power(float(base), -2.0 * (j + 1) / head_dim)
+
+
+def _attend_no_scale(q_rows, K, V, scale, visible):
+    return _orig_attend(q_rows, K, V, 1.0, visible)
+
+
+def _attend_off_by_one(q_rows, K, V, scale, visible):
+    return _orig_attend(q_rows, K, V, scale, np.maximum(np.asarray(visible) - 1, 1))
+
+
+def _attend_transposed(q_rows, K, V, scale, visible):
+    return _orig_attend(q_rows, V, K, scale, visible)
+
+
+def _bf16_truncate(x):
+    x = np.asarray(x, np.float64)
+    out = x.copy()
+    sel = np.isfinite(x) & (x != 0)
+    v = x[sel]
+    _, e = np.frexp(v)
+    sp = np.maximum(e - 8, -133)
+    out[sel] = np.ldexp(np.trunc(np.ldexp(v, -sp)), sp)
+    return out
+
+
+def _gather_mod_heads(cache, b, h, n, block_table=None):
+    return _orig_gather(cache, b, (h + 1) % cache.shape[1], n, block_table)
+
+
+_orig_attend = kv.attend
+_orig_rope = kv.rope
+_orig_gather = kv.gather_tokens
+
+MUTANTS = {
+    "rope_interleaved_pairs": ("rope", _rope_interleaved),
+    "rope_wrong_sign": ("rope", _rope_wrong_sign),
+    "rope_freq_index_off": ("rope_inv_freq", _inv_freq_off),
+    "attend_drops_scale": ("attend", _attend_no_scale),
+    "attend_mask_off_by_one": ("attend", _attend_off_by_one),
+    "attend_k_v_swapped": ("attend", _attend_transposed),
+    "bf16_truncates": ("bf16_round", _bf16_truncate),
+    "wrong_kv_head": ("gather_tokens", _gather_mod_heads),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_planted_mistake_is_caught(name, monkeypatch):
+    attr, fn = MUTANTS[name]
+    monkeypatch.setattr(kv, attr, fn)
+    failed = []
+    for pin in pins.ALL_PINS:
+        try:
+            pin(kv)
+        except (AssertionError, ValueError, IndexError):
+            failed.append(pin.__name__)
+    assert failed, f"no pin caught the planted mistake {name}"
