@@ -1,0 +1,434 @@
+"""Benchmark of one KV-cache decode step: RoPE + KV append + GQA flash decode.
+
+A step is one pass of the whole path over one batch: ``kv_append_rope``
+(rotate the new tokens, append k/v) followed by ``decode_attention[_paged]``
+(split-KV attention + log-sum-exp merge).  Inputs are resident in HBM before
+the timed region; the KV cache is larger than the 126 MB L2 for every default
+workload, so no flush is needed between steps (the tiny workload is flushed).
+``value`` is algorithmic bytes per step (see workloads.step_bytes) divided by
+the device time of the step, summed over ranks; ``e2e`` times the same step
+through the public API with the new tokens copied from pinned host memory and
+the output copied back, inside the timed region.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl ours|reference]
+
+Multi-GPU: one process per GPU (torchrun); every rank runs its own copy of the
+workload (independent sequences, no collective on the data path), so scaling
+is weak.  Times are device times (CUDA events), max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode-attention achieved HBM GB/s (% of B200 peak) and µs per decode step"
+FALLBACK_HBM_GBS = 6650.0
+L2_BYTES = 126 * 1024 * 1024
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="batched_gqa")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="CPU time budget of the oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def committed_traffic(workload: str):
+    """dram read+write bytes per decode launch from a committed ncu summary."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(workload)
+    if not e or e.get("stale"):
+        return None
+    return e.get("traffic_bytes_per_launch")
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting",
+    }
+
+    def __init__(self, index: int):
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # noqa: BLE001 - clocks are reported as unavailable
+            self.nvml = None
+        self.t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nvml.nvmlDeviceGetClockInfo(self.h, self.nvml.NVML_CLOCK_SM))
+                self.reasons |= self.nvml.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self.nvml:
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self.nvml:
+            self.t.join()
+
+    def summary(self):
+        if not self.nvml:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ CPU oracle
+_UNIT_POOL = {}
+
+
+def oracle_sample(w, seconds: float, seed: int):
+    """Time the fp64 oracle's decode on host cores over a bounded sample of the
+    workload: whole (sequence, kv head) units, one after another, until the
+    time budget is spent.  Returns (GB/s of attended K/V bytes, cores, text)."""
+    import numpy as np
+    import torch
+    import oracle
+    from kv_cache_decode_rope_b200.workloads import draw_lengths
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:  # noqa: BLE001
+        cores = 1
+    gen = torch.Generator().manual_seed(seed)
+    lens = draw_lengths(w, gen)
+    g, D, T = w.group, w.head_dim, w.q_len
+    key = (w.name, D, int(lens.max()) + T)
+    if key not in _UNIT_POOL:   # one stream of K/V rows, sliced per unit (drawn once, untimed)
+        rng = np.random.default_rng(seed)
+        n = key[2]
+        _UNIT_POOL[key] = (rng.standard_normal((n, D)).astype(np.float32).astype(np.float64),
+                           rng.standard_normal((n, D)).astype(np.float32).astype(np.float64))
+    K_all, V_all = _UNIT_POOL[key]
+    rng = np.random.default_rng(seed + 1)
+    done_bytes = 0
+    units = 0
+    elapsed = 0.0
+    while elapsed < seconds:
+        b = units % w.batch
+        L = int(lens[b])
+        n = L + T
+        K, V = K_all[:n], V_all[:n]
+        q = rng.standard_normal((T, g, D))
+        s0 = time.perf_counter()
+        for i in range(T):
+            oracle.attend(q[i], K, V, w.scale, [L + i + 1] * g)
+        elapsed += time.perf_counter() - s0
+        done_bytes += n * 2 * D * w.esize
+        units += 1
+    return done_bytes / elapsed / 1e9, cores, (
+        f"{units} (sequence, kv head) units of workload {w.name} (all {g * T} rows each), "
+        f"fp64 oracle attend, {elapsed:.1f} s of CPU time")
+
+
+# ------------------------------------------------------------------ GPU bench
+def run_ours(args, rank, world, local):
+    import torch
+    import kv_cache_decode_rope_b200 as kvd
+    from kv_cache_decode_rope_b200.workloads import WORKLOADS, make_inputs_device, step_bytes
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = WORKLOADS[args.workload]
+    if w.cache_mode == "prefill":
+        w = w.with_(cache_mode="random")
+    inp = make_inputs_device(w, seed=1000 + w.config_id + 7919 * rank, device=dev)
+    out_dtype = w.torch_dtype
+    out = torch.empty((w.batch, w.q_len, w.num_heads, w.head_dim), dtype=out_dtype, device=dev)
+    mkl = int(inp["seq_lens"].max()) + w.q_len
+    ws = torch.empty(kvd.workspace_size(batch=w.batch, num_heads=w.num_heads,
+                                        num_kv_heads=w.num_kv_heads, head_dim=w.head_dim,
+                                        q_len=w.q_len, dtype=w.torch_dtype),
+                     dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    bt = inp["block_table"]
+    nbytes = step_bytes(w, inp["seq_lens"].cpu(), torch.empty((), dtype=out_dtype).element_size())
+    cache_bytes = inp["k_cache"].numel() * inp["k_cache"].element_size() * 2
+    flush = cache_bytes < 2 * L2_BYTES
+    flush_buf = torch.empty(4 * L2_BYTES // 4, dtype=torch.int32, device=dev) if flush else None
+
+    def append(q, kn, vn, seq):
+        kvd.append_rope(q, kn, vn, inp["k_cache"], inp["v_cache"], seq, bt, rope_base=w.rope_base,
+                        status=status)
+
+    def decode(q, seq):
+        if bt is None:
+            kvd.decode_attention(q, inp["k_cache"], inp["v_cache"], seq, out, scale=w.scale,
+                                 max_kv_len=mkl, workspace=ws, status=status)
+        else:
+            kvd.decode_attention_paged(q, inp["k_cache"], inp["v_cache"], seq, bt, out, scale=w.scale,
+                                       max_kv_len=mkl, workspace=ws, status=status)
+
+    q, kn, vn, seq = inp["q"], inp["k_new"], inp["v_new"], inp["seq_lens"]
+    for _ in range(args.warmup):
+        append(q, kn, vn, seq)
+        decode(q, seq)
+    torch.cuda.synchronize()
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        t_all0 = torch.cuda.Event(enable_timing=True)
+        t_all1 = torch.cuda.Event(enable_timing=True)
+        t_all0.record()
+        for k in range(K):
+            if flush:
+                flush_buf.add_(1)
+            ev[k][0].record()
+            append(q, kn, vn, seq)
+            ev[k][1].record()
+            decode(q, seq)
+            ev[k][2].record()
+        t_all1.record()
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    step_ms = [ev[k][0].elapsed_time(ev[k][2]) for k in range(K)]
+    dec_ms = [ev[k][1].elapsed_time(ev[k][2]) for k in range(K)]
+    app_ms = [ev[k][0].elapsed_time(ev[k][1]) for k in range(K)]
+    total_ms = sum(step_ms) if flush else t_all0.elapsed_time(t_all1)
+    if status.item() != 0:
+        raise RuntimeError(f"device status flags set during the bench: {status.item()}")
+
+    # ---- end to end: pinned host inputs -> device, step, output -> host
+    hq = q.cpu().pin_memory()
+    hk = kn.cpu().pin_memory()
+    hv = vn.cpu().pin_memory()
+    hs = seq.cpu().pin_memory()
+    hbt = bt.cpu().pin_memory() if bt is not None else None
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    dq, dk, dv, ds = (torch.empty_like(t) for t in (q, kn, vn, seq))
+    dbt = torch.empty_like(bt) if bt is not None else None
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hs) + ((hbt,) if hbt is not None else ()))
+    d2h = hout.numel() * hout.element_size()
+
+    def e2e_step():
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        ds.copy_(hs, non_blocking=True)
+        if dbt is not None:
+            dbt.copy_(hbt, non_blocking=True)
+        kvd.append_rope(dq, dk, dv, inp["k_cache"], inp["v_cache"], ds, dbt, rope_base=w.rope_base)
+        if dbt is None:
+            kvd.decode_attention(dq, inp["k_cache"], inp["v_cache"], ds, out, scale=w.scale,
+                                 max_kv_len=mkl, workspace=ws)
+        else:
+            kvd.decode_attention_paged(dq, inp["k_cache"], inp["v_cache"], ds, dbt, out, scale=w.scale,
+                                       max_kv_len=mkl, workspace=ws)
+        hout.copy_(out, non_blocking=True)
+
+    for _ in range(max(3, args.warmup // 4)):
+        e2e_step()
+    torch.cuda.synchronize()
+    Ke = max(3, K // 4)
+    if world > 1:
+        torch.distributed.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(Ke):
+        if flush:
+            flush_buf.add_(1)
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / Ke
+
+    res = dict(total_ms=total_ms, step_ms=statistics.median(step_ms),
+               mean_step_ms=total_ms / K, dec_ms=sum(dec_ms) / K, dec_med=statistics.median(dec_ms),
+               app_ms=sum(app_ms) / K, e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, bytes=nbytes,
+               clocks=clk.summary(), flush=flush, cache_bytes=cache_bytes, w=w, mkl=mkl)
+    return res
+
+
+def reduce_max(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def workload_config(w, extra=None):
+    c = {"workload": w.name, "batch": w.batch, "num_heads": w.num_heads, "num_kv_heads": w.num_kv_heads,
+         "head_dim": w.head_dim, "q_len": w.q_len,
+         "cache": f"paged (page {w.page_size})" if w.paged else "contiguous",
+         "cache_len": w.cache_len if w.cache_len is not None else f"log-uniform {w.len_range}"}
+    if extra:
+        c.update(extra)
+    return c
+
+
+def main():
+    args = parse()
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        return main_reference(args, rank, world)
+    import torch
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    r = run_ours(args, rank, world, local)
+    w = r["w"]
+    K = args.steps
+    total_ms = reduce_max(r["total_ms"], world)
+    dec_ms = reduce_max(r["dec_ms"], world)
+    e2e_ms = reduce_max(r["e2e_ms"], world)
+    ms_step = total_ms / K
+    step_bytes = r["bytes"]["step"]
+    value = world * step_bytes / (ms_step * 1e-3) / 1e9
+    peak, peak_kind = measured_peaks()
+    dec_gbs = r["bytes"]["decode"] / (dec_ms * 1e-3) / 1e9
+    traffic = committed_traffic(w.name)
+    line = {
+        "metric": METRIC,
+        "value": round(value, 1),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 5),
+        "us_per_step": round(ms_step * 1e3, 2),
+        "pct_of_peak": round(100 * value / world / peak, 1),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if w.dtype == "bf16" else "f32",
+        "data": "synthetic (seeded N(0,1) cache, shapes of the workload)",
+        "config": workload_config(w, {
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "l2": ("flushed between steps" if r["flush"] else
+                   f"inputs larger than L2 ({r['cache_bytes'] / 2**20:.0f} MiB KV cache)"),
+            "step": "kv_append_rope + decode_attention" + ("_paged" if w.paged else ""),
+            "max_kv_len": r["mkl"]}),
+        "roofline": {
+            "bound": "hbm",
+            "kernel": "decode_attention (split-KV kernel + LSE merge)",
+            "achieved": round(dec_gbs, 1),
+            "peak": peak,
+            "peak_source": f"{peak_kind} hbm_gbs",
+            "unit": "GB/s",
+            "frac": round(dec_gbs / peak, 4),
+            "us_per_launch": round(dec_ms * 1e3, 2),
+            "algorithmic_bytes_per_launch": r["bytes"]["decode"],
+            "traffic": traffic,
+        },
+        "append_us": round(r["app_ms"] * 1e3, 2),
+        "e2e": {"value": round(world * step_bytes / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+                "us_per_step": round(e2e_ms * 1e3, 2),
+                "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
+        "gpu_launches": 3 * K,
+        "clocks": r["clocks"],
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        v, cores, sample = oracle_sample(w, args.cpu_seconds, seed=1000 + w.config_id)
+        line["cpu_baseline"] = {"value": round(v, 4), "unit": "GB/s", "cores": cores,
+                                "kind": "oracle", "sample": sample}
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main_reference(args, rank, world):
+    """The oracle as it stands, timed on the host cores (rank 0 only)."""
+    if rank != 0:
+        return 0
+    from kv_cache_decode_rope_b200.workloads import WORKLOADS, step_bytes, draw_lengths
+    import torch
+    w = WORKLOADS[args.workload]
+    if w.cache_mode == "prefill":
+        w = w.with_(cache_mode="random")
+    # bounded: the whole run stays near two minutes of CPU work whatever K is
+    per_step = min(1.0, 120.0 / max(1, args.steps + args.warmup))
+    vals = []
+    info = None
+    for k in range(args.warmup + args.steps):
+        v, cores, sample = oracle_sample(w, per_step, seed=1000 + w.config_id + k)
+        if k >= args.warmup:
+            vals.append(v)
+            info = (cores, sample)
+    value = statistics.median(vals)
+    lens = draw_lengths(w, torch.Generator().manual_seed(1000 + w.config_id))
+    step_b = step_bytes(w, lens, w.esize)["step"]
+    ms = step_b / (value * 1e9) * 1e3
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic", "config": workload_config(w),
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": info[0], "kind": "oracle",
+                         "sample": "each step: " + info[1]},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

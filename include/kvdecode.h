@@ -1,0 +1,189 @@
+/*
+ * kvdecode.h -- C ABI of the KV-cache decode-step library (sm_100a).
+ *
+ * One autoregressive decode step of a transformer attention layer:
+ *   1. kv_append_rope: rotate the new tokens' q and k with RoPE at their
+ *      absolute positions and append k and v to the layer's KV cache;
+ *   2. decode_attention / decode_attention_paged: attend every new query
+ *      token, with grouped-query heads, against the whole cache.
+ * The result equals the last rows of a full, non-cached causal attention over
+ * the prefix (ferric-core 0.1.0, examples/generate.rs: module doc comment and
+ * the exactness check in `run`).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - All tensor pointers are DEVICE pointers owned by the caller.  The library
+ *   allocates nothing, keeps no per-call state, never synchronises the
+ *   stream, and may be called from several host threads at once.
+ * - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ * - Host-side argument checks run before any launch; a failed check returns a
+ *   negative kvd_status and launches nothing.  A launch failure returns
+ *   KVD_ERR_CUDA (details via cudaGetLastError in the caller's runtime).
+ * - Problems only the device can see (a block-table entry outside
+ *   [0, num_pages), a length beyond the cache capacity, a pipeline wait that
+ *   ran out of its iteration limit) skip the affected access and OR a
+ *   KVD_FLAG_* bit into *params->status when that pointer is non-NULL.  No
+ *   kernel traps or asserts.
+ *
+ * Notation: B = batch, T = q_len (new tokens per sequence), Hq / Hkv = query /
+ * key-value heads, g = Hq / Hkv, D = head_dim, L_b = seq_lens[b] = tokens
+ * already cached for sequence b BEFORE the step.  New token i of sequence b
+ * sits at absolute position L_b + i and attends positions 0 .. L_b + i.
+ * Query head h reads kv head h / g.
+ *
+ * Layouts (row-major, innermost last):
+ *   q, out          [B, T, Hq, D]
+ *   k_new, v_new    [B, T, Hkv, D]
+ *   contiguous cache  k_cache, v_cache [B, Hkv, max_seq_len, D]
+ *   paged cache       k_cache, v_cache [num_pages, Hkv, page_size, D]
+ *   block_table     [B, max_pages_per_seq] int32: logical page j of sequence b
+ *                   (positions j*page_size .. ) lives in physical page
+ *                   block_table[b*max_pages_per_seq + j]
+ *   seq_lens        [B] int32
+ * Every pointer must be 16-byte aligned.
+ */
+#ifndef KVDECODE_H
+#define KVDECODE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KVD_API __attribute__((visibility("default")))
+#else
+#define KVD_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum kvd_status {
+  KVD_OK = 0,
+  KVD_ERR_INVALID_ARG = -1, /* null pointer, bad size, bad alignment        */
+  KVD_ERR_UNSUPPORTED = -2, /* valid request outside the compiled kernels   */
+  KVD_ERR_WORKSPACE = -3,   /* workspace NULL or smaller than required      */
+  KVD_ERR_CUDA = -4         /* launch failure or no usable device           */
+} kvd_status;
+
+typedef enum kvd_dtype {
+  KVD_F32 = 0,
+  KVD_BF16 = 1
+} kvd_dtype;
+
+/* Bits OR-ed into *kvd_params.status by the device. */
+#define KVD_FLAG_PAGE_OUT_OF_RANGE 0x1 /* block-table entry outside [0, num_pages) */
+#define KVD_FLAG_CAPACITY 0x2          /* L_b + T beyond the cache capacity        */
+#define KVD_FLAG_WAIT_TIMEOUT 0x4      /* a pipeline wait hit its iteration limit  */
+
+/* Parameters shared by all entry points.  Fields a call does not use are
+ * ignored (e.g. rope_base by the attention calls, paging fields by the
+ * contiguous calls). */
+typedef struct kvd_params {
+  int batch;             /* B >= 1                                                    */
+  int num_heads;         /* Hq >= 1                                                   */
+  int num_kv_heads;      /* Hkv >= 1, Hq % Hkv == 0                                   */
+  int head_dim;          /* D: 16, 32, 64, 128 or 256                                 */
+  int q_len;             /* T >= 1 new tokens per sequence                            */
+  float scale;           /* softmax scale applied to q.k (e.g. 1/sqrt(D))             */
+  float rope_base;       /* RoPE base (e.g. 10000); kv_append_rope only               */
+  int dtype;             /* kvd_dtype of q, k_new, v_new and both caches              */
+  int out_dtype;         /* kvd_dtype of out                                          */
+  int max_seq_len;       /* contiguous: token capacity per (sequence, kv head)        */
+  int page_size;         /* paged: tokens per page, a positive multiple of 16         */
+  int num_pages;         /* paged: pages in the pool                                  */
+  int max_pages_per_seq; /* paged: block_table row stride                             */
+  int max_kv_len;        /* attention: host upper bound on L_b + T over the batch     */
+  int* status;           /* optional device int, OR-ed with KVD_FLAG_* bits; may be 0 */
+} kvd_params;
+
+/*
+ * kv_append_rope -- RoPE on the new tokens and KV-cache append.
+ *
+ * Defined by ferric-core 0.1.0, examples/generate.rs, `step_gpu`: the new
+ * token's q and k are rotated with `rope_off_t` at the absolute position, v is
+ * not rotated, and k and v are appended to the cache (`kc.extend`,
+ * `vc.extend`).  Batched with a per-sequence position as in the
+ * ferrum-sampler 0.7.0 README, "Key Optimizations" ("Batched RoPE: per-item
+ * positions in single kernel launch").
+ *
+ * RoPE reading (the pages do not fix the pairing): half-split pairs (j, j+D/2)
+ * for j < D/2 are rotated by angle (L_b+i) * rope_base^(-2j/D):
+ *   (a, b) -> (a cos - b sin, a sin + b cos).
+ * The angle and the rotation are evaluated in fp64 and rounded once to dtype
+ * (round to nearest even).
+ *
+ * q        in/out [B,T,Hq,D]: rotated in place.
+ * k_new    in [B,T,Hkv,D]; v_new in [B,T,Hkv,D] (not modified).
+ * k_cache, v_cache: receive rotated k and v at position L_b + i; no other slot
+ *          is written.
+ * block_table: NULL selects the contiguous layout (max_seq_len used);
+ *          otherwise the paged layout (page_size, num_pages,
+ *          max_pages_per_seq used).  The caller must have mapped every page
+ *          that positions L_b .. L_b+T-1 fall in.
+ * seq_lens: read only; the caller advances it after the step.
+ * Returns KVD_OK or a negative kvd_status.
+ */
+KVD_API int kv_append_rope(const kvd_params* p, void* q, const void* k_new, const void* v_new,
+                   void* k_cache, void* v_cache, const int32_t* seq_lens,
+                   const int32_t* block_table, void* stream);
+
+/*
+ * decode_attention -- grouped-query attention of the T new query tokens
+ * against the contiguous cache.
+ *
+ * Defined by ferric-core 0.1.0, examples/generate.rs, `step_gpu`
+ * (`mha_decode_t(q1, kc, vc, h, h, dh, s)`: single-query attention over all
+ * cached tokens, with separate q-head and kv-head counts) and `cpu::mha_causal`
+ * in `layer_cpu` (causal softmax attention).  Long contexts are split over
+ * several CTAs and merged by log-sum-exp, the split-K scheme named
+ * "Flash Decoding" in the ferrum-sampler 0.7.0 README, "Key Optimizations".
+ *
+ * q        in [B,T,Hq,D], already rotated (kv_append_rope writes it).
+ * k_cache, v_cache in [B,Hkv,max_seq_len,D]: positions 0 .. L_b+T-1 are read.
+ * seq_lens in [B]: L_b (tokens before the step); the new tokens are the last T
+ *          of the L_b+T attended positions, with a causal mask among them.
+ * out      out [B,T,Hq,D] in out_dtype:
+ *          out = sum_t softmax_t(scale * q.k_t) v_t over the visible t.
+ * workspace: caller-owned device scratch of at least
+ *          kvd_workspace_size(p) bytes (split partials); contents need no
+ *          initialisation and are overwritten.  Two calls that run at the
+ *          same time must not share a workspace.
+ * Requires max_kv_len >= L_b + T for every b (the grid is sized from it).
+ */
+KVD_API int decode_attention(const kvd_params* p, const void* q, const void* k_cache,
+                     const void* v_cache, const int32_t* seq_lens, void* out,
+                     void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * decode_attention_paged -- decode_attention over the paged cache.
+ *
+ * Block-table indirection into a shared page pool, as in the ferrum-sampler
+ * 0.7.0 README, "Key Optimizations" ("Paged KV attention: GPU block pool with
+ * block-table indirection").  Same arguments and result as decode_attention;
+ * k_cache/v_cache are [num_pages, Hkv, page_size, D] and block_table maps
+ * logical pages to physical pages.
+ */
+KVD_API int decode_attention_paged(const kvd_params* p, const void* q, const void* k_cache,
+                           const void* v_cache, const int32_t* seq_lens,
+                           const int32_t* block_table, void* out, void* workspace,
+                           size_t workspace_bytes, void* stream);
+
+/*
+ * kvd_workspace_size -- bytes of workspace decode_attention[_paged] needs for
+ * these parameters (depends on batch, heads, q_len, head_dim; not on the
+ * device).  Returns 0 if the parameters are invalid.
+ */
+KVD_API size_t kvd_workspace_size(const kvd_params* p);
+
+/* kvd_status_string -- static, human-readable text for a kvd_status value. */
+KVD_API const char* kvd_status_string(int status);
+
+/* kvd_version -- library version as 10000*major + 100*minor + patch. */
+KVD_API int kvd_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVDECODE_H */

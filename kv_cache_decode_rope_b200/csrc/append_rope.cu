@@ -1,0 +1,156 @@
+// Kernel A: RoPE on the new tokens + KV-cache append (contiguous or paged).
+//
+// ferric-core 0.1.0, examples/generate.rs, `step_gpu`: the new token's q and k
+// are rotated at the absolute position (`rope_off_t`), v is not, and k and v
+// are appended to the per-layer cache (`kc.extend`, `vc.extend`).  As in the
+// ferrum-sampler 0.7.0 README ("Batched RoPE: per-item positions in single
+// kernel launch") every sequence of the batch carries its own position.
+//
+// One CTA per new token (b, i).  The CTA first evaluates the D/2 rotation
+// angles pos * base^(-2j/D) and their sine/cosine in fp64 into shared memory
+// (positions reach 1e5+, where an fp32 angle would be off by ~1e-2 rad).  Each
+// thread then rotates EPV half-split pairs (j, j + D/2) of one head row with
+// 16-byte loads and stores, in fp64, rounding once to the storage type, and
+// copies 16-byte pieces of v.  q is rotated in place; k and v go to the slot
+// of position seq_lens[b] + i.
+#include <cuda_bf16.h>
+
+#include "kvd_device.cuh"
+#include "kvd_internal.h"
+
+namespace kvd {
+namespace {
+
+template <typename T>
+struct Conv;
+template <>
+struct Conv<float> {
+  __device__ static double to_d(float x) { return (double)x; }
+  __device__ static float from_d(double x) { return __double2float_rn(x); }
+};
+template <>
+struct Conv<__nv_bfloat16> {
+  __device__ static double to_d(__nv_bfloat16 x) { return (double)__bfloat162float(x); }
+  __device__ static __nv_bfloat16 from_d(double x) { return __double2bfloat16(x); }
+};
+
+template <typename T, int D>
+__global__ void __launch_bounds__(256) append_rope_kernel(AppendArgs a) {
+  constexpr int EPV = 16 / (int)sizeof(T);  // elements per 16-byte vector
+  constexpr int HALF = D / 2;
+  constexpr int TPR = HALF / EPV;           // threads per rotated head row
+  constexpr int VPR = D / EPV;              // 16-byte vectors per head row
+  static_assert(HALF % EPV == 0, "half head must hold whole vectors");
+
+  __shared__ double s_cos[HALF];
+  __shared__ double s_sin[HALF];
+
+  const int b = blockIdx.x / a.T;
+  const int i = blockIdx.x % a.T;
+  const long long pos = (long long)a.seq_lens[b] + i;
+
+  for (int j = threadIdx.x; j < HALF; j += blockDim.x) {
+    const double inv_freq = pow(a.rope_base, -2.0 * (double)j / (double)D);
+    double s, c;
+    sincos((double)pos * inv_freq, &s, &c);
+    s_cos[j] = c;
+    s_sin[j] = s;
+  }
+
+  // Where position `pos` of sequence b lives; -1 if it is outside the cache.
+  long long slot_base = -1;  // element offset of (kv head 0, pos); heads are `head_stride` apart
+  long long head_stride = 0;
+  if (pos >= 0) {
+    if (a.block_table == nullptr) {
+      if (pos < a.max_seq_len) {
+        slot_base = ((long long)b * a.Hkv * a.max_seq_len + pos) * D;
+        head_stride = (long long)a.max_seq_len * D;
+      }
+    } else {
+      const long long lp = pos / a.page_size;
+      if (lp < a.max_pages_per_seq) {
+        const int page = a.block_table[(long long)b * a.max_pages_per_seq + lp];
+        if (page >= 0 && page < a.num_pages) {
+          slot_base = ((long long)page * a.Hkv * a.page_size + pos % a.page_size) * D;
+          head_stride = (long long)a.page_size * D;
+        } else if (threadIdx.x == 0 && a.status) {
+          atomicOr(a.status, KVD_FLAG_PAGE_OUT_OF_RANGE);
+        }
+      }
+    }
+  }
+  if (slot_base < 0 && threadIdx.x == 0 && a.status) atomicOr(a.status, KVD_FLAG_CAPACITY);
+  __syncthreads();
+
+  const long long tok = (long long)b * a.T + i;
+  const int n_rot = (a.Hq + a.Hkv) * TPR;
+  const int n_v = a.Hkv * VPR;
+  for (int w = threadIdx.x; w < n_rot + n_v; w += blockDim.x) {
+    if (w < n_rot) {
+      const int row = w / TPR;
+      const int j0 = (w % TPR) * EPV;
+      const T* src;
+      T* dst;
+      if (row < a.Hq) {
+        T* qrow = reinterpret_cast<T*>(a.q) + (tok * a.Hq + row) * D;
+        src = qrow;
+        dst = qrow;
+      } else {
+        const int hk = row - a.Hq;
+        src = reinterpret_cast<const T*>(a.k_new) + (tok * a.Hkv + hk) * D;
+        if (slot_base < 0) continue;
+        dst = reinterpret_cast<T*>(a.k_cache) + slot_base + hk * head_stride;
+      }
+      const uint4 ua = *reinterpret_cast<const uint4*>(src + j0);
+      const uint4 ub = *reinterpret_cast<const uint4*>(src + HALF + j0);
+      const T* xa = reinterpret_cast<const T*>(&ua);
+      const T* xb = reinterpret_cast<const T*>(&ub);
+      uint4 ra, rb;
+      T* ya = reinterpret_cast<T*>(&ra);
+      T* yb = reinterpret_cast<T*>(&rb);
+#pragma unroll
+      for (int e = 0; e < EPV; ++e) {
+        const double c = s_cos[j0 + e], s = s_sin[j0 + e];
+        const double va = Conv<T>::to_d(xa[e]), vb = Conv<T>::to_d(xb[e]);
+        // explicit roundings: a*c - b*s and a*s + b*c, each product rounded
+        ya[e] = Conv<T>::from_d(__dsub_rn(__dmul_rn(va, c), __dmul_rn(vb, s)));
+        yb[e] = Conv<T>::from_d(__dadd_rn(__dmul_rn(va, s), __dmul_rn(vb, c)));
+      }
+      *reinterpret_cast<uint4*>(dst + j0) = ra;
+      *reinterpret_cast<uint4*>(dst + HALF + j0) = rb;
+    } else {
+      if (slot_base < 0) continue;
+      const int w2 = w - n_rot;
+      const int hk = w2 / VPR;
+      const int part = (w2 % VPR) * EPV;
+      const T* src = reinterpret_cast<const T*>(a.v_new) + (tok * a.Hkv + hk) * D + part;
+      T* dst = reinterpret_cast<T*>(a.v_cache) + slot_base + hk * head_stride + part;
+      *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
+    }
+  }
+}
+
+template <typename T>
+cudaError_t launch_t(const AppendArgs& a, cudaStream_t st) {
+  const int grid = a.B * a.T;
+  const int work = (a.Hq + a.Hkv) * a.D / 2 + a.Hkv * a.D;  // upper bound on items
+  int threads = 32;
+  while (threads < 256 && threads < work / (16 / (int)sizeof(T))) threads *= 2;
+  switch (a.D) {
+    case 16: append_rope_kernel<T, 16><<<grid, threads, 0, st>>>(a); break;
+    case 32: append_rope_kernel<T, 32><<<grid, threads, 0, st>>>(a); break;
+    case 64: append_rope_kernel<T, 64><<<grid, threads, 0, st>>>(a); break;
+    case 128: append_rope_kernel<T, 128><<<grid, threads, 0, st>>>(a); break;
+    case 256: append_rope_kernel<T, 256><<<grid, threads, 0, st>>>(a); break;
+    default: return cudaErrorNotSupported;
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_append(const AppendArgs& a, int bf16, cudaStream_t st) {
+  return bf16 ? launch_t<__nv_bfloat16>(a, st) : launch_t<float>(a, st);
+}
+
+}  // namespace kvd

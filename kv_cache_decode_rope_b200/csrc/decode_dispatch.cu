@@ -1,0 +1,33 @@
+// Host dispatch of the split-KV decode over storage type and cache layout.
+#include "kvd_internal.h"
+
+namespace kvd {
+
+cudaError_t launch_decode_bf16_contig(const DecodeArgs& a, cudaStream_t st);
+cudaError_t launch_decode_bf16_paged(const DecodeArgs& a, cudaStream_t st);
+cudaError_t launch_decode_f32_contig(const DecodeArgs& a, cudaStream_t st);
+cudaError_t launch_decode_f32_paged(const DecodeArgs& a, cudaStream_t st);
+
+bool decode_supported(int D, int bf16, int R) {
+  if (R < 1 || R > kMaxRows) return false;
+  if (D == 16 || D == 32 || D == 64 || D == 128) return true;
+  return D == 256 && bf16;
+}
+
+int decode_grid(int B, int Hkv, int max_kv_len, int num_sms) {
+  const long long chunks = (long long)B * Hkv * ((max_kv_len + kChunk - 1) / kChunk);
+  long long g = (chunks + 3) / 4;  // at least one 64-token stage per CTA
+  const long long cap = (long long)2 * num_sms;
+  if (g > cap) g = cap;
+  if (g > kMaxGrid) g = kMaxGrid;
+  if (g < 1) g = 1;
+  return (int)g;
+}
+
+cudaError_t launch_decode(const DecodeArgs& a, int bf16, cudaStream_t st) {
+  if (a.block_table)
+    return bf16 ? launch_decode_bf16_paged(a, st) : launch_decode_f32_paged(a, st);
+  return bf16 ? launch_decode_bf16_contig(a, st) : launch_decode_f32_contig(a, st);
+}
+
+}  // namespace kvd

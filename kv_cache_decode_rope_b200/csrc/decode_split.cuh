@@ -1,0 +1,654 @@
+// Kernels B and C: split-KV flash decode over a contiguous or paged KV cache,
+// and the log-sum-exp merge of the splits.
+//
+// What is computed: ferric-core 0.1.0, examples/generate.rs, `step_gpu`
+// (`mha_decode_t`: the new query attends every cached token) with the causal
+// rule of `cpu::mha_causal` among several new tokens, grouped-query heads as
+// in ferrox-models' `decoder` (q head h reads kv head h / g).  Work is split
+// along the cache ("Flash Decoding: split-K for long-context decode", and one
+// launch for all batch items, "Batched attention kernel", ferrum-sampler 0.7.0
+// README, Key Optimizations) and merged by log-sum-exp.
+//
+// B200 design (not the pages' design; they describe other hardware):
+// * Work quantum = 16 cached tokens of one (sequence, kv head) "unit".  The
+//   chunks of all units are laid end to end and cut into `grid` equal ranges,
+//   one per CTA, so ragged batches balance exactly and every SM streams the
+//   same number of bytes.  Grid = a multiple of the SM count.
+// * One CTA owns all g*q_len query rows of a unit, so each K/V byte leaves
+//   HBM once.  A producer warp streams K and V stages (64 tokens of D=128
+//   bf16 = 16 KB each) into shared memory with 1-D bulk copies (one per
+//   page-slice for the paged layout) into a 3-deep mbarrier ring.
+// * Consumer warps: each lane owns 16 bytes of a token row (8 bf16 dims) and
+//   the matching slice of every query row, held in fp32 registers.  q.k partial
+//   sums over the lane's dims are reduced across the lanes of a token with a
+//   "transpose-reduce" (each shuffle level halves the values a lane keeps), so
+//   one shuffle per score replaces log2(lanes) per score.  Packed fp32 FMA
+//   (two lanes of work per instruction) does both contractions.  Online softmax
+//   in base 2 with the scale folded into q.
+// * A CTA whose range covers a whole unit writes `out`; otherwise it writes a
+//   normalised partial (o, lse) to the workspace slot (cta + unit), and
+//   kernel C merges the partials of each unit.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+
+#include "kvd_device.cuh"
+#include "kvd_internal.h"
+
+namespace kvd {
+namespace {
+
+__host__ __device__ constexpr int ilog2(int x) { return x <= 1 ? 0 : 1 + ilog2(x / 2); }
+__host__ __device__ constexpr int cmin(int a, int b) { return a < b ? a : b; }
+__host__ __device__ constexpr int cmax(int a, int b) { return a > b ? a : b; }
+
+template <typename T, int D>
+struct Geo {
+  static constexpr int ES = (int)sizeof(T);
+  static constexpr int EPV = 16 / ES;             // elements per lane vector
+  static constexpr int NP = EPV / 2;              // fp32 pairs per vector
+  static constexpr int LPT = D / EPV;             // lanes per token row
+  static constexpr int TPP = 32 / LPT;            // tokens per warp pass
+  static constexpr int TOKEN_BYTES = D * ES;
+  static constexpr int STAGE_TOKENS = cmax(kChunk, cmin(128, 16384 / TOKEN_BYTES));
+  static constexpr int STAGE_CHUNKS = STAGE_TOKENS / kChunk;
+  static constexpr int STAGE_BYTES = STAGE_TOKENS * TOKEN_BYTES;
+  static constexpr int NSTAGES = 3;
+  static_assert(LPT >= 1 && LPT <= 32, "a token row must fit one warp");
+};
+
+// Shared-memory carve-up (bytes), identical on host and device.
+template <typename T, int D, int RPW, int NTW>
+struct Smem {
+  using G = Geo<T, D>;
+  static constexpr int TW_TOKENS = G::STAGE_TOKENS / NTW;
+  static constexpr int TB = cmin(cmin(32 / RPW, TW_TOKENS / G::TPP), G::LPT);
+  static constexpr int P_FLOATS = TB * G::TPP * RPW;  // p buffer per warp
+  __host__ __device__ static size_t stages() { return (size_t)2 * G::NSTAGES * G::STAGE_BYTES; }
+  __host__ __device__ static size_t bars_off() { return stages(); }
+  __host__ __device__ static size_t p_off() { return bars_off() + 2 * G::NSTAGES * 8; }
+  __host__ __device__ static size_t comb_off(int ncw) { return p_off() + (size_t)ncw * P_FLOATS * 4; }
+  __host__ __device__ static size_t ml_off(int ncw) { return comb_off(ncw) + (size_t)ncw * RPW * D * 4; }
+  __host__ __device__ static size_t prefix_off(int ncw) { return ml_off(ncw) + (size_t)ncw * RPW * 2 * 4; }
+  __host__ __device__ static size_t total(int ncw, int B) {
+    return prefix_off(ncw) + (size_t)(B + 1) * 4;
+  }
+};
+
+struct SegState {
+  int b, hk;         // unit
+  int k0;            // first chunk of the unit in this CTA's range
+  long long x;       // global chunk index of k0
+};
+
+// Per-sequence attended length N_b = L_b + T, clamped to the capacity.
+__device__ __forceinline__ int attended_len(const DecodeArgs& a, int b, bool flag) {
+  long long L = a.seq_lens[b];
+  long long N = L + a.T;
+  if (L < 0 || N > a.cap_tokens) {
+    if (flag && a.status) atomicOr(a.status, KVD_FLAG_CAPACITY);
+    N = L < 0 ? a.T : (long long)a.cap_tokens;
+    if (N > a.cap_tokens) N = a.cap_tokens;
+  }
+  return (int)N;
+}
+
+template <typename T, int D, int RPW, int NTW, bool PAGED>
+__global__ void __launch_bounds__(NTW == 1 ? 288 : 160)
+    decode_kernel(DecodeArgs a, int nrg) {
+  using G = Geo<T, D>;
+  using S = Smem<T, D, RPW, NTW>;
+  using VT = VecTraits<T>;
+  constexpr int EPV = G::EPV, NP = G::NP, LPT = G::LPT, TPP = G::TPP;
+  constexpr int TB = S::TB;
+  constexpr int NV = TB * RPW;  // q.k partial sums per lane per block
+  constexpr int TW_TOKENS = S::TW_TOKENS;
+  constexpr int NBLK = TW_TOKENS / (TB * TPP);
+  constexpr int LOG_LPT = ilog2(LPT);
+  constexpr int KLEV = cmin(LOG_LPT, ilog2(NV));  // transposing shuffle levels
+  constexpr int NOWN = NV >> KLEV;                 // scores a lane ends with
+  constexpr int SHIFT = LOG_LPT - KLEV;            // low lane bits that only replicate
+  static_assert(NV * TPP * NBLK * NTW == RPW * G::STAGE_TOKENS, "block tiling");
+  static_assert(NOWN <= RPW, "each lane's scores must belong to distinct rows");
+
+  extern __shared__ __align__(128) unsigned char smem[];
+  const int ncw = nrg * NTW;                 // consumer warps
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  T* sK = reinterpret_cast<T*>(smem);
+  T* sV = reinterpret_cast<T*>(smem + (size_t)G::NSTAGES * G::STAGE_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::bars_off());
+  uint64_t* empty = full + G::NSTAGES;
+  float* sP = reinterpret_cast<float*>(smem + S::p_off());
+  float* sComb = reinterpret_cast<float*>(smem + S::comb_off(ncw));
+  float* sML = reinterpret_cast<float*>(smem + S::ml_off(ncw));
+  int* sPrefix = reinterpret_cast<int*>(smem + S::prefix_off(ncw));
+
+  // ---- prologue: clear stages, barriers, per-sequence chunk prefix --------
+  {
+    uint4* z = reinterpret_cast<uint4*>(smem);
+    const int n16 = (int)(S::stages() / 16);
+    for (int k = threadIdx.x; k < n16; k += blockDim.x) z[k] = make_uint4(0, 0, 0, 0);
+  }
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < G::NSTAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], ncw);
+    }
+  }
+  {
+    // block-wide exclusive scan of chunks per sequence: sPrefix[b] = sum_{b'<b} n_b'
+    const int nthr = blockDim.x;
+    const int per = (a.B + nthr - 1) / nthr;
+    const int lo = threadIdx.x * per;
+    const int hi = min(a.B, lo + per);
+    int tsum = 0;
+    for (int b = lo; b < hi; ++b) tsum += (attended_len(a, b, blockIdx.x == 0) + kChunk - 1) / kChunk;
+    int incl = tsum;
+#pragma unroll
+    for (int m = 1; m < 32; m <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, m);
+      if (lane >= m) incl += v;
+    }
+    int* sWarpTot = reinterpret_cast<int*>(sML);  // scratch before first use of sML
+    if (lane == 31) sWarpTot[warp] = incl;
+    __syncthreads();
+    int woff = 0;
+    for (int w = 0; w < warp; ++w) woff += sWarpTot[w];
+    int run = woff + incl - tsum;
+    for (int b = lo; b < hi; ++b) {
+      sPrefix[b] = run;
+      run += (attended_len(a, b, false) + kChunk - 1) / kChunk;
+    }
+    if (hi == a.B && lo < hi) sPrefix[a.B] = run;
+    __syncthreads();
+  }
+  fence_barrier_init();
+  fence_proxy_async_smem();
+  __syncthreads();
+
+  const long long total = (long long)a.Hkv * sPrefix[a.B];
+  if (blockIdx.x == 0 && threadIdx.x == 0) *a.total_chunks = total;
+  const long long x0 = total * blockIdx.x / a.grid;
+  const long long x1 = total * (blockIdx.x + 1) / a.grid;
+  if (x0 >= x1) return;  // empty range: no copies issued, nothing to write
+
+  // locate the unit holding chunk x0: largest b with Hkv * prefix[b] <= x0
+  SegState st;
+  {
+    int lo = 0, hi = a.B - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if ((long long)a.Hkv * sPrefix[mid] <= x0) lo = mid; else hi = mid - 1;
+    }
+    st.b = lo;
+    const int nb = sPrefix[lo + 1] - sPrefix[lo];
+    const long long r = x0 - (long long)a.Hkv * sPrefix[lo];
+    st.hk = (int)(r / nb);
+    st.k0 = (int)(r % nb);
+    st.x = x0;
+  }
+
+  if (warp == ncw) {
+    // ======================= producer warp ===============================
+    int s = 0;
+    bool failed = false;
+    SegState p = st;
+    while (p.x < x1 && !failed) {
+      const int nb = sPrefix[p.b + 1] - sPrefix[p.b];
+      const int Nb = attended_len(a, p.b, false);
+      const int kend = (int)min((long long)nb, p.k0 + (x1 - p.x));
+      for (int kk = p.k0; kk < kend; kk += G::STAGE_CHUNKS, ++s) {
+        const int slot = s % G::NSTAGES;
+        const uint32_t par = (uint32_t)(s / G::NSTAGES) & 1u;
+        // one lane waits, the warp follows its verdict (keeps the warp converged)
+        int ok = 1;
+        if (lane == 0) ok = mbar_wait(&empty[slot], par ^ 1u, a.status) ? 1 : 0;
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) { failed = true; break; }
+        const int nck = min(G::STAGE_CHUNKS, kend - kk);
+        const int t0 = kk * kChunk;
+        T* dK = sK + (size_t)slot * G::STAGE_TOKENS * D;
+        T* dV = sV + (size_t)slot * G::STAGE_TOKENS * D;
+        if constexpr (!PAGED) {
+          const int ntok = min(nck * kChunk, Nb - t0);
+          const uint32_t bytes = (uint32_t)ntok * G::TOKEN_BYTES;
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&full[slot], 2 * bytes);
+            const size_t off = (((size_t)p.b * a.Hkv + p.hk) * a.max_seq_len + t0) * D;
+            bulk_g2s(dK, reinterpret_cast<const T*>(a.k_cache) + off, bytes, &full[slot]);
+            bulk_g2s(dV, reinterpret_cast<const T*>(a.v_cache) + off, bytes, &full[slot]);
+          }
+        } else {
+          // lane c < nck copies chunk c of the stage (16 tokens inside one page)
+          uint32_t bytes = 0;
+          size_t off = 0;
+          if (lane < nck) {
+            const int tc = t0 + lane * kChunk;
+            const int ntok = min(kChunk, Nb - tc);
+            const int lp = tc / a.page_size;
+            const int page = a.block_table[(size_t)p.b * a.max_pages_per_seq + lp];
+            if (page >= 0 && page < a.num_pages) {
+              bytes = (uint32_t)ntok * G::TOKEN_BYTES;
+              off = (((size_t)page * a.Hkv + p.hk) * a.page_size + (tc % a.page_size)) * D;
+            } else if (a.status) {
+              atomicOr(a.status, KVD_FLAG_PAGE_OUT_OF_RANGE);
+            }
+          }
+          uint32_t tot = bytes;
+#pragma unroll
+          for (int m = 16; m >= 1; m >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, m);
+          if (lane == 0) mbar_arrive_expect_tx(&full[slot], 2 * tot);
+          __syncwarp();
+          if (bytes) {
+            bulk_g2s(dK + (size_t)lane * kChunk * D, reinterpret_cast<const T*>(a.k_cache) + off,
+                     bytes, &full[slot]);
+            bulk_g2s(dV + (size_t)lane * kChunk * D, reinterpret_cast<const T*>(a.v_cache) + off,
+                     bytes, &full[slot]);
+          }
+        }
+        __syncwarp();
+      }
+      p.x += kend - p.k0;
+      p.k0 = 0;
+      if (++p.hk == a.Hkv) { p.hk = 0; ++p.b; }
+    }
+    // drain: every issued copy lands before the CTA may exit
+    if (lane == 0) {
+      for (int k = max(0, s - G::NSTAGES); k < s; ++k)
+        if (!mbar_wait(&full[k % G::NSTAGES], (uint32_t)(k / G::NSTAGES) & 1u, a.status)) break;
+    }
+    return;
+  }
+
+  // ========================= consumer warps ==============================
+  const int rg = warp / NTW;             // row group
+  const int tw = warp % NTW;             // token slice of each stage
+  const int hg = lane / LPT;             // token within a warp pass
+  const int lg = lane % LPT;             // 16-byte slice of the head dim
+  const int ncons = ncw * 32;
+  // rows of this lane's own scores (fixed for the kernel)
+  int own_row[NOWN];
+#pragma unroll
+  for (int i = 0; i < NOWN; ++i) own_row[i] = (i + NOWN * (lg >> SHIFT)) % RPW;
+  int own_tok[NOWN];  // token index within a block (0..TB-1) of own score i
+#pragma unroll
+  for (int i = 0; i < NOWN; ++i) own_tok[i] = (i + NOWN * (lg >> SHIFT)) / RPW;
+  float* myP = sP + warp * S::P_FLOATS;
+
+  int s = 0;
+  bool failed = false;
+  SegState c = st;
+  while (c.x < x1) {
+    const int nb = sPrefix[c.b + 1] - sPrefix[c.b];
+    const int Nb = attended_len(a, c.b, false);
+    const int Lb = Nb - a.T;  // first new-token position (may be <= 0 after clamping)
+    const int kend = (int)min((long long)nb, c.k0 + (x1 - c.x));
+    const int u = c.b * a.Hkv + c.hk;
+
+    // -- segment init: q rows of this warp, pre-scaled for exp2
+    float2 q2[RPW][NP];
+    float2 o2[RPW][NP];
+    float m_all[RPW];
+    float m_own[NOWN], l_own[NOWN];
+    int vis_own[NOWN];  // visible token count of own rows
+#pragma unroll
+    for (int r = 0; r < RPW; ++r) {
+      const int rglob = rg * RPW + r;
+      m_all[r] = -INFINITY;
+#pragma unroll
+      for (int e = 0; e < NP; ++e) { o2[r][e] = make_float2(0.f, 0.f); q2[r][e] = make_float2(0.f, 0.f); }
+      if (rglob < a.R) {
+        const int i = rglob / a.g;
+        const int h = c.hk * a.g + rglob % a.g;
+        const T* qp = reinterpret_cast<const T*>(a.q) + (((size_t)c.b * a.T + i) * a.Hq + h) * D + lg * EPV;
+        float2 f[NP];
+        VT::unpack(*reinterpret_cast<const uint4*>(qp), f);
+#pragma unroll
+        for (int e = 0; e < NP; ++e) q2[r][e] = make_float2(f[e].x * a.qscale, f[e].y * a.qscale);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < NOWN; ++i) {
+      m_own[i] = -INFINITY;
+      l_own[i] = 0.f;
+      const int rglob = rg * RPW + own_row[i];
+      vis_own[i] = (rglob < a.R) ? Lb + rglob / a.g + 1 : Nb;
+    }
+
+    for (int kk = c.k0; kk < kend; kk += G::STAGE_CHUNKS, ++s) {
+      const int slot = s % G::NSTAGES;
+      const uint32_t par = (uint32_t)(s / G::NSTAGES) & 1u;
+      if (!failed && !mbar_wait(&full[slot], par, a.status)) failed = true;
+      const int t0 = kk * kChunk;
+      const int nvalid = min(min(G::STAGE_CHUNKS, kend - kk) * kChunk, Nb - t0);
+      // masking is needed when the stage is short or reaches the new tokens
+      const bool tail = (nvalid < G::STAGE_TOKENS) || (t0 + G::STAGE_TOKENS > Lb + 1);
+      const T* Ks = sK + (size_t)slot * G::STAGE_TOKENS * D;
+      const T* Vs = sV + (size_t)slot * G::STAGE_TOKENS * D;
+
+#pragma unroll 1
+      for (int blk = 0; blk < NBLK; ++blk) {
+        const int tbase = tw * TW_TOKENS + blk * TB * TPP;  // first token of the block in the stage
+        // ---- scores: partial dot products over this lane's dims
+        float sc[NV];
+#pragma unroll
+        for (int j = 0; j < TB; ++j) {
+          const int t = tbase + j * TPP + hg;
+          float2 kf[NP];
+          VT::unpack(*reinterpret_cast<const uint4*>(Ks + (size_t)t * D + lg * EPV), kf);
+#pragma unroll
+          for (int r = 0; r < RPW; ++r) {
+            float2 acc = fmul2(q2[r][0], kf[0]);
+#pragma unroll
+            for (int e = 1; e < NP; ++e) acc = ffma2(q2[r][e], kf[e], acc);
+            sc[j * RPW + r] = acc.x + acc.y;
+          }
+        }
+        // ---- transpose-reduce across the LPT lanes of a token
+        {
+          int n = NV;
+#pragma unroll
+          for (int lev = 0; lev < LOG_LPT; ++lev) {
+            const int m = LPT >> (lev + 1);
+            if (lev < KLEV) {
+              const bool upper = (lane & m) != 0;
+              const int half = NV >> (lev + 1);
+#pragma unroll
+              for (int i2 = 0; i2 < half; ++i2) {
+                const float lo_v = sc[i2], hi_v = sc[i2 + half];
+                const float send = upper ? lo_v : hi_v;
+                const float keep = upper ? hi_v : lo_v;
+                sc[i2] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+              }
+            } else {
+              sc[0] += __shfl_xor_sync(0xffffffffu, sc[0], m);
+            }
+          }
+          (void)n;
+        }
+        // ---- mask
+        if (tail) {
+#pragma unroll
+          for (int i = 0; i < NOWN; ++i) {
+            const int t = tbase + own_tok[i] * TPP + hg;
+            if (t >= nvalid || t0 + t >= vis_own[i]) sc[i] = -INFINITY;
+          }
+        }
+        // ---- block max per own row, across lanes holding the same row
+        float bm[NOWN];
+#pragma unroll
+        for (int i = 0; i < NOWN; ++i) bm[i] = sc[i];
+#pragma unroll
+        for (int m = 1; m < 32; m <<= 1) {
+          bool same_row;
+          if (m >= LPT) same_row = true;
+          else if (m < (1 << SHIFT)) same_row = false;  // replica lanes hold equal values
+          else same_row = ((NOWN * (m >> SHIFT)) % RPW) == 0;
+          if (same_row) {
+#pragma unroll
+            for (int i = 0; i < NOWN; ++i) bm[i] = fmaxf(bm[i], __shfl_xor_sync(0xffffffffu, bm[i], m));
+          }
+        }
+        // ---- every row's block max to every lane; rescale accumulators
+#pragma unroll
+        for (int r = 0; r < RPW; ++r) {
+          const float bmr = __shfl_sync(0xffffffffu, bm[r % NOWN], (r / NOWN) << SHIFT);
+          const float mn = fmaxf(m_all[r], bmr);
+          const float ms = (mn == -INFINITY) ? 0.f : mn;
+          const float alpha = fast_exp2(m_all[r] - ms);
+          m_all[r] = mn;
+          const float2 al = make_float2(alpha, alpha);
+#pragma unroll
+          for (int e = 0; e < NP; ++e) o2[r][e] = fmul2(o2[r][e], al);
+        }
+        // ---- probabilities of own scores
+#pragma unroll
+        for (int i = 0; i < NOWN; ++i) {
+          const float mn = fmaxf(m_own[i], bm[i]);
+          const float ms = (mn == -INFINITY) ? 0.f : mn;
+          const float pr = fast_exp2(sc[i] - ms);
+          l_own[i] = l_own[i] * fast_exp2(m_own[i] - ms) + pr;
+          m_own[i] = mn;
+          myP[(own_tok[i] * TPP + hg) * RPW + own_row[i]] = pr;
+        }
+        __syncwarp();
+        // ---- o += p v
+#pragma unroll
+        for (int j = 0; j < TB; ++j) {
+          const int t = tbase + j * TPP + hg;
+          float2 vf[NP];
+          VT::unpack(*reinterpret_cast<const uint4*>(Vs + (size_t)t * D + lg * EPV), vf);
+          const float* pj = myP + (j * TPP + hg) * RPW;
+          float pv[RPW];
+          if constexpr (RPW % 4 == 0) {
+#pragma unroll
+            for (int r4 = 0; r4 < RPW; r4 += 4) {
+              const float4 v4 = *reinterpret_cast<const float4*>(pj + r4);
+              pv[r4] = v4.x; pv[r4 + 1] = v4.y; pv[r4 + 2] = v4.z; pv[r4 + 3] = v4.w;
+            }
+          } else {
+#pragma unroll
+            for (int r = 0; r < RPW; ++r) pv[r] = pj[r];
+          }
+#pragma unroll
+          for (int r = 0; r < RPW; ++r) {
+            const float2 pp = make_float2(pv[r], pv[r]);
+#pragma unroll
+            for (int e = 0; e < NP; ++e) o2[r][e] = ffma2(pp, vf[e], o2[r][e]);
+          }
+        }
+        __syncwarp();
+      }
+      if (lane == 0) mbar_arrive(&empty[slot]);
+    }
+
+    // -- segment end: reduce within the warp, then across token slices
+#pragma unroll
+    for (int m = 1; m < 32; m <<= 1) {
+      bool same_row;
+      if (m >= LPT) same_row = true;
+      else if (m < (1 << SHIFT)) same_row = false;
+      else same_row = ((NOWN * (m >> SHIFT)) % RPW) == 0;
+      if (same_row) {
+#pragma unroll
+        for (int i = 0; i < NOWN; ++i) l_own[i] += __shfl_xor_sync(0xffffffffu, l_own[i], m);
+      }
+    }
+#pragma unroll
+    for (int m = LPT; m < 32; m <<= 1) {
+#pragma unroll
+      for (int r = 0; r < RPW; ++r)
+#pragma unroll
+        for (int e = 0; e < NP; ++e) {
+          o2[r][e].x += __shfl_xor_sync(0xffffffffu, o2[r][e].x, m);
+          o2[r][e].y += __shfl_xor_sync(0xffffffffu, o2[r][e].y, m);
+        }
+    }
+    if (lane < LPT) {
+#pragma unroll
+      for (int r = 0; r < RPW; ++r) {
+        float* dst = sComb + ((size_t)warp * RPW + r) * D + lg * EPV;
+#pragma unroll
+        for (int e = 0; e < NP; ++e) { dst[2 * e] = o2[r][e].x; dst[2 * e + 1] = o2[r][e].y; }
+      }
+      if ((lg & ((1 << SHIFT) - 1)) == 0) {
+#pragma unroll
+        for (int i = 0; i < NOWN; ++i) {
+          if (own_tok[i] == 0) {
+            sML[((size_t)warp * RPW + own_row[i]) * 2 + 1] = l_own[i];
+          }
+        }
+      }
+    }
+    if (lane == 0) {
+#pragma unroll
+      for (int r = 0; r < RPW; ++r) sML[((size_t)warp * RPW + r) * 2] = m_all[r];
+    }
+    named_bar_sync(1, ncons);
+
+    const bool whole = (c.k0 == 0) && (kend == nb);
+    const long long slot_idx = (long long)blockIdx.x + u;
+    for (int e = threadIdx.x; e < nrg * RPW * D; e += ncons) {
+      const int rgi = e / (RPW * D);
+      const int r = (e / D) % RPW;
+      const int d = e % D;
+      const int rglob = rgi * RPW + r;
+      if (rglob >= a.R) continue;
+      float M = -INFINITY;
+      for (int w = 0; w < NTW; ++w) M = fmaxf(M, sML[((size_t)(rgi * NTW + w) * RPW + r) * 2]);
+      const float Ms = (M == -INFINITY) ? 0.f : M;
+      float L = 0.f, O = 0.f;
+      for (int w = 0; w < NTW; ++w) {
+        const int ww = rgi * NTW + w;
+        const float wt = fast_exp2(sML[((size_t)ww * RPW + r) * 2] - Ms);
+        L += wt * sML[((size_t)ww * RPW + r) * 2 + 1];
+        O += wt * sComb[((size_t)ww * RPW + r) * D + d];
+      }
+      const float o = (L > 0.f) ? O / L : 0.f;
+      if (whole) {
+        const int i = rglob / a.g;
+        const int h = c.hk * a.g + rglob % a.g;
+        const size_t oi = (((size_t)c.b * a.T + i) * a.Hq + h) * D + d;
+        if (a.out_bf16) reinterpret_cast<__nv_bfloat16*>(a.out)[oi] = __float2bfloat16_rn(o);
+        else reinterpret_cast<float*>(a.out)[oi] = o;
+      } else {
+        a.part_o[((size_t)slot_idx * a.R + rglob) * D + d] = o;
+        if (d == 0) a.part_lse[(size_t)slot_idx * a.R + rglob] = (L > 0.f) ? Ms + fast_log2(L) : -INFINITY;
+      }
+    }
+    if (threadIdx.x == 0) {
+      if (c.k0 == 0) a.unit_ctas[u].x = blockIdx.x;
+      if (kend == nb) a.unit_ctas[u].y = blockIdx.x;
+    }
+    named_bar_sync(1, ncons);
+
+    c.x += kend - c.k0;
+    c.k0 = 0;
+    if (++c.hk == a.Hkv) { c.hk = 0; ++c.b; }
+  }
+}
+
+// Kernel C: one warp per (unit, row) merges the partials of units split over
+// several CTAs: out = sum_s 2^(lse_s - LSE) o_s with LSE = log2 sum_s 2^lse_s.
+template <int D>
+__global__ void __launch_bounds__(256) combine_kernel(DecodeArgs a) {
+  constexpr int PER = (D + 31) / 32;
+  const long long wid = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const long long U = (long long)a.B * a.Hkv;
+  if (wid >= U * a.R) return;
+  const int u = (int)(wid / a.R);
+  const int r = (int)(wid % a.R);
+  const int2 cr = a.unit_ctas[u];
+  if (cr.x >= cr.y) return;  // one CTA covered the unit and wrote out directly
+  // CTAs whose chunk range came out empty wrote no partial: skip them
+  const long long total = *a.total_chunks;
+  auto nonempty = [&](int c) {
+    return total * c / a.grid < total * (c + 1) / a.grid;
+  };
+  float M = -INFINITY;
+  for (int c = cr.x; c <= cr.y; ++c)
+    if (nonempty(c)) M = fmaxf(M, a.part_lse[((size_t)c + u) * a.R + r]);
+  const float Ms = (M == -INFINITY) ? 0.f : M;
+  float acc[PER];
+#pragma unroll
+  for (int k = 0; k < PER; ++k) acc[k] = 0.f;
+  float L = 0.f;
+  for (int c = cr.x; c <= cr.y; ++c) {
+    if (!nonempty(c)) continue;
+    const size_t sl = (size_t)c + u;
+    const float w = fast_exp2(a.part_lse[sl * a.R + r] - Ms);
+    L += w;
+    const float* po = a.part_o + (sl * a.R + r) * D;
+#pragma unroll
+    for (int k = 0; k < PER; ++k) {
+      const int d = lane + 32 * k;
+      if (d < D) acc[k] += w * po[d];
+    }
+  }
+  const int b = u / a.Hkv, hk = u % a.Hkv;
+  const int i = r / a.g;
+  const int h = hk * a.g + r % a.g;
+  const size_t ob = (((size_t)b * a.T + i) * a.Hq + h) * D;
+  const float inv = (L > 0.f) ? 1.f / L : 0.f;
+#pragma unroll
+  for (int k = 0; k < PER; ++k) {
+    const int d = lane + 32 * k;
+    if (d < D) {
+      const float o = acc[k] * inv;
+      if (a.out_bf16) reinterpret_cast<__nv_bfloat16*>(a.out)[ob + d] = __float2bfloat16_rn(o);
+      else reinterpret_cast<float*>(a.out)[ob + d] = o;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- host side
+inline int d_index(int D) {
+  return D == 16 ? 0 : D == 32 ? 1 : D == 64 ? 2 : D == 128 ? 3 : D == 256 ? 4 : -1;
+}
+
+// Per (D, row config): devices on which the shared-memory opt-in was set.
+template <typename T, bool PAGED>
+std::atomic<unsigned long long>& smem_attr_flag(int di, int cfg) {
+  static std::atomic<unsigned long long> flags[5][6];
+  return flags[di][cfg];
+}
+
+template <typename T, int D, int RPW, int NTW, bool PAGED>
+cudaError_t launch_one(const DecodeArgs& a, int nrg, int cfg_idx, cudaStream_t st) {
+  using S = Smem<T, D, RPW, NTW>;
+  const int ncw = nrg * NTW;
+  const size_t smem = S::total(ncw, a.B);
+  if (smem > 227 * 1024) return cudaErrorNotSupported;
+  auto kern = decode_kernel<T, D, RPW, NTW, PAGED>;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  auto& flag = smem_attr_flag<T, PAGED>(d_index(D), cfg_idx);
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (!(flag.load() & bit)) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+    if (e != cudaSuccess) return e;
+    flag.fetch_or(bit);
+  }
+  kern<<<a.grid, (ncw + 1) * 32, smem, st>>>(a, nrg);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const long long warps = (long long)a.B * a.Hkv * a.R;
+  const int cblocks = (int)((warps * 32 + 255) / 256);
+  combine_kernel<D><<<cblocks, 256, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+template <typename T, int D, bool PAGED>
+cudaError_t launch_rows(const DecodeArgs& a, cudaStream_t st) {
+  if (a.R <= 1) return launch_one<T, D, 1, 4, PAGED>(a, 1, 0, st);
+  if (a.R <= 2) return launch_one<T, D, 2, 4, PAGED>(a, 1, 1, st);
+  if (a.R <= 4) return launch_one<T, D, 4, 4, PAGED>(a, 1, 2, st);
+  if (a.R <= 8) return launch_one<T, D, 8, 4, PAGED>(a, 1, 3, st);
+  if (a.R <= 16) return launch_one<T, D, 8, 2, PAGED>(a, 2, 4, st);
+  if (a.R <= kMaxRows) return launch_one<T, D, 8, 1, PAGED>(a, (a.R + 7) / 8, 5, st);
+  return cudaErrorNotSupported;
+}
+
+}  // namespace
+
+template <typename T, bool PAGED>
+cudaError_t launch_decode_t(const DecodeArgs& a, cudaStream_t st) {
+  switch (a.D) {
+    case 16: return launch_rows<T, 16, PAGED>(a, st);
+    case 32: return launch_rows<T, 32, PAGED>(a, st);
+    case 64: return launch_rows<T, 64, PAGED>(a, st);
+    case 128: return launch_rows<T, 128, PAGED>(a, st);
+    case 256:
+      if constexpr (sizeof(T) == 2) return launch_rows<T, 256, PAGED>(a, st);
+      else return cudaErrorNotSupported;
+    default: return cudaErrorNotSupported;
+  }
+}
+
+}  // namespace kvd

@@ -1,0 +1,66 @@
+// Internal launch interface between the C-ABI layer (kvd_api.cu) and the
+// kernel translation units.  Not part of the public ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/kvdecode.h"
+
+namespace kvd {
+
+constexpr int kChunk = 16;        // tokens per work quantum (one page of 16, or a slice of one)
+constexpr int kMaxGrid = 1024;    // upper bound on decode CTAs; sizes the workspace
+constexpr int kMaxRows = 64;      // g * q_len rows per (sequence, kv head) on the CUDA-core path
+constexpr int kMaxBatch = 8192;   // sequences per call (per-CTA length scan lives in shared memory)
+
+struct AppendArgs {
+  void* q;
+  const void* k_new;
+  const void* v_new;
+  void* k_cache;
+  void* v_cache;
+  const int32_t* seq_lens;
+  const int32_t* block_table;  // null: contiguous
+  int* status;
+  int B, T, Hq, Hkv, D;
+  int max_seq_len;
+  int page_size, num_pages, max_pages_per_seq;
+  double rope_base;
+};
+
+struct DecodeArgs {
+  const void* q;
+  const void* k_cache;
+  const void* v_cache;
+  const int32_t* seq_lens;
+  const int32_t* block_table;  // null: contiguous
+  void* out;
+  float* part_o;      // [slots, R, D]
+  float* part_lse;    // [slots, R]
+  int2* unit_ctas;    // [U]: first and last CTA that touched each (sequence, kv head)
+  long long* total_chunks;  // written by CTA 0: chunks over all units (defines every CTA's range)
+  int* status;
+  int B, T, Hq, Hkv, g, R, D;
+  int max_seq_len;                       // contiguous capacity
+  int page_size, num_pages, max_pages_per_seq;
+  int cap_tokens;                        // capacity per sequence in tokens
+  float qscale;                          // scale * log2(e)
+  int out_bf16;
+  int grid;                              // decode CTAs
+};
+
+// Workspace carve-up, shared by kvd_workspace_size and the launch.
+struct WorkspaceLayout {
+  size_t unit_ctas_off, total_off, part_lse_off, part_o_off, total;
+};
+WorkspaceLayout workspace_layout(int B, int Hkv, int R, int D);
+
+cudaError_t launch_append(const AppendArgs& a, int bf16, cudaStream_t st);
+// Returns cudaErrorNotSupported when no kernel is compiled for the shape.
+cudaError_t launch_decode(const DecodeArgs& a, int bf16, cudaStream_t st);
+int decode_grid(int B, int Hkv, int max_kv_len, int num_sms);
+bool decode_supported(int D, int bf16, int R);
+
+}  // namespace kvd

@@ -214,3 +214,82 @@ def logical_kv(inp: dict, b: int, h: int, n: int, which: str = "k") -> torch.Ten
         page = int(bt[b, t0 // P])
         rows.append(cache[page, h, :min(P, n - t0)])
     return torch.cat(rows, 0)
+
+
+def make_inputs_device(w: Workload, seed: int, device="cuda") -> dict:
+    """The same layout and distributions as ``make_inputs``, drawn directly on
+    the device with a seeded CUDA generator (used for timing, where copying
+    gigabytes from the host would only slow set-up).  Unused cache slots are
+    zero.  Lengths and the page permutation are drawn on the host as in
+    ``make_inputs``."""
+    hgen = torch.Generator().manual_seed(seed)
+    dgen = torch.Generator(device=device).manual_seed(seed)
+    B, Hq, Hkv, D, T = w.batch, w.num_heads, w.num_kv_heads, w.head_dim, w.q_len
+    dt = w.torch_dtype
+    lens = draw_lengths(w, hgen)
+
+    def draw(shape):
+        if w.dist == "uniform":
+            return torch.rand(shape, generator=dgen, device=device) * 0.2 - 0.1
+        return torch.randn(shape, generator=dgen, device=device)
+
+    out = {"workload": w, "seed": seed, "seq_lens": lens.to(torch.int32).to(device)}
+    out["q"] = draw((B, T, Hq, D)).to(dt)
+    out["k_new"] = draw((B, T, Hkv, D)).to(dt)
+    out["v_new"] = draw((B, T, Hkv, D)).to(dt)
+    P = w.page_size
+    if w.paged:
+        pages_per_seq = [(int(L) + T + P - 1) // P for L in lens]
+        num_pages = sum(pages_per_seq)
+        perm = torch.randperm(num_pages, generator=hgen).to(torch.int32)
+        bt = torch.full((B, max(pages_per_seq)), -1, dtype=torch.int32)
+        off = 0
+        for b, n in enumerate(pages_per_seq):
+            bt[b, :n] = perm[off:off + n]
+            off += n
+        k_cache = torch.zeros((num_pages, Hkv, P, D), dtype=dt, device=device)
+        v_cache = torch.zeros_like(k_cache)
+        out.update(block_table=bt.to(device), num_pages=num_pages, max_pages_per_seq=bt.shape[1])
+    else:
+        cap = round_up(int(lens.max()) + T, 16)
+        k_cache = torch.zeros((B, Hkv, cap, D), dtype=dt, device=device)
+        v_cache = torch.zeros_like(k_cache)
+        out.update(block_table=None, max_seq_len=cap)
+    for b in range(B):
+        L = int(lens[b])
+        for h in range(Hkv):
+            k = draw((L, D))
+            v = draw((L, D))
+            if w.peaked_frac > 0:
+                n_peak = int(math.floor(w.peaked_frac * L))
+                idx = torch.randperm(L, generator=dgen, device=device)[:n_peak]
+                k[idx] *= w.peaked_scale
+            if w.paged:
+                t = torch.arange(L, device=device)
+                pages = out["block_table"][b, t // P].long()
+                k_cache[pages, h, t % P] = k.to(dt)
+                v_cache[pages, h, t % P] = v.to(dt)
+            else:
+                k_cache[b, h, :L] = k.to(dt)
+                v_cache[b, h, :L] = v.to(dt)
+    out["k_cache"] = k_cache
+    out["v_cache"] = v_cache
+    return out
+
+
+def step_bytes(w: Workload, seq_lens, out_esize: int) -> dict:
+    """Algorithmic bytes one decode step must move (the unit of the GB/s
+    figures).  ``decode``: every attended K and V row once, q read, out
+    written.  ``append``: q read + written, k_new and v_new read, k and v
+    written to the cache, the length (and page) indices read."""
+    lens = [int(x) for x in seq_lens]
+    B, T, Hq, Hkv, D, es = w.batch, w.q_len, w.num_heads, w.num_kv_heads, w.head_dim, w.esize
+    kv = sum(L + T for L in lens) * Hkv * 2 * D * es
+    q = B * T * Hq * D * es
+    out = B * T * Hq * D * out_esize
+    idx = B * 4
+    if w.paged:
+        idx += sum((L + T + w.page_size - 1) // w.page_size for L in lens) * 4
+    decode = kv + q + out + idx
+    append = 2 * q + 4 * B * T * Hkv * D * es + B * 4 + (B * T * 4 if w.paged else 0)
+    return {"decode": decode, "append": append, "step": decode + append, "kv": kv}

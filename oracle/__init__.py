@@ -14,5 +14,6 @@ from .kv_decode import (  # noqa: F401
     max_abs_diff,
     rope,
     rope_inv_freq,
+    rotate_new_tokens,
     round_store,
 )

@@ -117,6 +117,18 @@ def _slot(b, p, cache_shape, block_table, page_size):
     return int(block_table[b, p // page_size]), p % page_size
 
 
+def rotate_new_tokens(q, k_new, v_new, seq_lens, base: float, dtype: str):
+    """q and k of the new tokens rotated at positions seq_lens[b] + i, and v,
+    each rounded to the storage dtype: ``(q_rot, k_rot, v_stored)``."""
+    q = np.asarray(q, F64)
+    T = q.shape[1]
+    pos = np.asarray(seq_lens, dtype=np.int64)[:, None] + np.arange(T)[None, :]  # [B, T]
+    q_rot = round_store(rope(q, pos[:, :, None], base), dtype)
+    k_rot = round_store(rope(np.asarray(k_new, F64), pos[:, :, None], base), dtype)
+    v_st = round_store(np.asarray(v_new, F64), dtype)
+    return q_rot, k_rot, v_st
+
+
 def append_rope(q, k_new, v_new, k_cache, v_cache, seq_lens, base: float,
                 dtype: str, block_table=None):
     """Rotate q and k_new at positions seq_lens[b] + i, store k and v.
@@ -134,9 +146,7 @@ def append_rope(q, k_new, v_new, k_cache, v_cache, seq_lens, base: float,
     Hkv = k_new.shape[2]
     page_size = kc.shape[2] if block_table is not None else None
     pos = np.asarray(seq_lens, dtype=np.int64)[:, None] + np.arange(T)[None, :]  # [B, T]
-    q_rot = round_store(rope(q, pos[:, :, None], base), dtype)
-    k_rot = round_store(rope(k_new, pos[:, :, None], base), dtype)
-    v_st = round_store(v_new, dtype)
+    q_rot, k_rot, v_st = rotate_new_tokens(q, k_new, v_new, seq_lens, base, dtype)
     for b in range(B):
         for i in range(T):
             p = int(pos[b, i])
