@@ -12,6 +12,15 @@ BF16_TOL = 2e-3     # max |gpu - oracle| with bf16 inputs (the exactness bound o
 F32_TOL = 1e-5      # fp32 inputs
 
 
+def log_error(tag: str, value: float) -> None:
+    """Append a measured error to $KVD_ERROR_LOG (if set) for the design notes."""
+    import os
+    path = os.environ.get("KVD_ERROR_LOG")
+    if path:
+        with open(path, "a") as f:
+            f.write(f"{tag}\t{value:.3e}\n")
+
+
 def np64(t: torch.Tensor) -> np.ndarray:
     return t.detach().cpu().float().numpy().astype(np.float64)
 
