@@ -65,15 +65,29 @@ def measured_peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
+def kernel_source_hash() -> str:
+    """Hash of the CUDA sources; a committed ncu figure is only valid for it."""
+    import glob
+    import hashlib
+    d = os.path.join(ROOT, "kv_cache_decode_rope_b200", "csrc")
+    files = sorted(glob.glob(os.path.join(d, "*.cu*"))) + sorted(glob.glob(os.path.join(d, "*.h")))
+    h = hashlib.sha256()
+    for f in files:
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
 def committed_traffic(workload: str):
-    """dram read+write bytes per decode launch from a committed ncu summary."""
+    """dram read+write bytes per decode launch from a committed ncu summary,
+    or None when the kernels changed since that capture."""
     p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         d = json.load(f)
     e = d.get(workload)
-    if not e or e.get("stale"):
+    if not e or e.get("source_hash") != kernel_source_hash():
         return None
     return e.get("traffic_bytes_per_launch")
 
