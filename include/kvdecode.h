@@ -176,6 +176,37 @@ KVD_API int decode_attention_paged(const kvd_params* p, const void* q, const voi
  */
 KVD_API size_t kvd_workspace_size(const kvd_params* p);
 
+/*
+ * decode_attention_static -- decode_attention / decode_attention_paged for
+ * callers that cannot allocate device memory.
+ *
+ * The pages have no counterpart of this call; it exists for callers that have
+ * no way to provide a workspace: code running inside a host framework that
+ * owns all device memory and hands none out after start-up, a latency-
+ * critical path where an allocation would synchronise the device, or a
+ * foreign-function caller without a device allocator.
+ *
+ * Same inputs, outputs and result as decode_attention (block_table == NULL)
+ * or decode_attention_paged (block_table != NULL).  Instead of a caller
+ * workspace it uses a scratch array of KVD_STATIC_WORKSPACE_BYTES compiled
+ * into the library: every GPU that loads the library holds that array until
+ * the process exits.  The call allocates nothing.
+ * - The first call on a device looks up the array's device address and the
+ *   SM count (once per device, with that device current); make that first
+ *   call before any stream capture.
+ * - All calls on a device share the one array and it keeps the last call's
+ *   contents; no part of it needs clearing (every word a call reads is
+ *   written earlier in the same call).  Calls that overlap on the GPU (other
+ *   streams, other host threads) race on it: serialise them.
+ * - Returns KVD_ERR_WORKSPACE when the problem needs more scratch than the
+ *   array holds (about (2 * SMs + B * Hkv) * g * q_len * (head_dim + 1) * 4
+ *   bytes); other errors as for decode_attention.
+ */
+#define KVD_STATIC_WORKSPACE_BYTES (16u << 20)
+KVD_API int decode_attention_static(const kvd_params* p, const void* q, const void* k_cache,
+                                    const void* v_cache, const int32_t* seq_lens,
+                                    const int32_t* block_table, void* out, void* stream);
+
 /* kvd_status_string -- static, human-readable text for a kvd_status value. */
 KVD_API const char* kvd_status_string(int status);
 

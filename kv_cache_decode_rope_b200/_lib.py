@@ -23,6 +23,8 @@ KVD_FLAG_PAGE_OUT_OF_RANGE = 0x1
 KVD_FLAG_CAPACITY = 0x2
 KVD_FLAG_WAIT_TIMEOUT = 0x4
 
+KVD_STATIC_WORKSPACE_BYTES = 16 << 20
+
 # Every exported symbol of include/kvdecode.h with its ctypes signature.
 c_int, c_size_t, c_void_p, c_char_p = ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_char_p
 
@@ -57,6 +59,8 @@ SIGNATURES = {
                                  c_size_t, c_void_p]),
     "decode_attention_paged": (c_int, [PP, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                        c_void_p, c_void_p, c_size_t, c_void_p]),
+    "decode_attention_static": (c_int, [PP, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                        c_void_p, c_void_p]),
     "kvd_workspace_size": (c_size_t, [PP]),
     "kvd_status_string": (c_char_p, [c_int]),
     "kvd_version": (c_int, []),
