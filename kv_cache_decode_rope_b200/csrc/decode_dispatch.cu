@@ -8,16 +8,25 @@ cudaError_t launch_decode_bf16_paged(const DecodeArgs& a, cudaStream_t st);
 cudaError_t launch_decode_f32_contig(const DecodeArgs& a, cudaStream_t st);
 cudaError_t launch_decode_f32_paged(const DecodeArgs& a, cudaStream_t st);
 
+cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t st);
+
+bool use_tensor_cores(int D, int bf16, int R) { return bf16 && D == 128 && R >= kTcMinRows; }
+
 bool decode_supported(int D, int bf16, int R) {
-  if (R < 1 || R > kMaxRows) return false;
+  if (R < 1) return false;
+  if (use_tensor_cores(D, bf16, R)) return R <= kMaxRows;
+  if (R > kMaxRowsCore) return false;
   if (D == 16 || D == 32 || D == 64 || D == 128) return true;
   return D == 256 && bf16;
 }
 
-int decode_grid(int B, int Hkv, int max_kv_len, int num_sms) {
+// CTAs of the decode launch: one per SM for the tensor-core kernel (its
+// shared memory fills an SM), two per SM for the CUDA-core kernel, never
+// more than one 64-token stage of work per CTA below that.
+int decode_grid(int B, int Hkv, int max_kv_len, int num_sms, int D, int bf16, int R) {
   const long long chunks = (long long)B * Hkv * ((max_kv_len + kChunk - 1) / kChunk);
   long long g = (chunks + 3) / 4;  // at least one 64-token stage per CTA
-  const long long cap = (long long)2 * num_sms;
+  const long long cap = (long long)(use_tensor_cores(D, bf16, R) ? 1 : 2) * num_sms;
   if (g > cap) g = cap;
   if (g > kMaxGrid) g = kMaxGrid;
   if (g < 1) g = 1;
@@ -25,6 +34,7 @@ int decode_grid(int B, int Hkv, int max_kv_len, int num_sms) {
 }
 
 cudaError_t launch_decode(const DecodeArgs& a, int bf16, cudaStream_t st) {
+  if (use_tensor_cores(a.D, bf16, a.R)) return launch_decode_tc(a, st);
   if (a.block_table)
     return bf16 ? launch_decode_bf16_paged(a, st) : launch_decode_f32_paged(a, st);
   return bf16 ? launch_decode_bf16_contig(a, st) : launch_decode_f32_contig(a, st);

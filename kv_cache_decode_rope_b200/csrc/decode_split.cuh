@@ -96,6 +96,54 @@ __device__ __forceinline__ int attended_len(const DecodeArgs& a, int b, bool fla
   return (int)N;
 }
 
+// Block-wide exclusive scan of chunks per sequence: sPrefix[b] = sum over
+// b' < b of ceil(N_b' / 16), sPrefix[B] = total.  All threads of the block
+// call it; `scratch` holds one int per warp.  Ends with __syncthreads.
+__device__ __forceinline__ void chunk_prefix_scan(const DecodeArgs& a, int* sPrefix, int* scratch) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nthr = blockDim.x;
+  const int per = (a.B + nthr - 1) / nthr;
+  const int lo = threadIdx.x * per;
+  const int hi = min(a.B, lo + per);
+  int tsum = 0;
+  for (int b = lo; b < hi; ++b) tsum += (attended_len(a, b, blockIdx.x == 0) + kChunk - 1) / kChunk;
+  int incl = tsum;
+#pragma unroll
+  for (int m = 1; m < 32; m <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, m);
+    if (lane >= m) incl += v;
+  }
+  if (lane == 31) scratch[warp] = incl;
+  __syncthreads();
+  int woff = 0;
+  for (int w = 0; w < warp; ++w) woff += scratch[w];
+  int run = woff + incl - tsum;
+  for (int b = lo; b < hi; ++b) {
+    sPrefix[b] = run;
+    run += (attended_len(a, b, false) + kChunk - 1) / kChunk;
+  }
+  if (hi == a.B && lo < hi) sPrefix[a.B] = run;
+  __syncthreads();
+}
+
+// The unit (sequence b, kv head hk) and chunk within it of global chunk x:
+// largest b with Hkv * prefix[b] <= x, then the head and chunk inside b.
+__device__ __forceinline__ SegState locate_chunk(const DecodeArgs& a, const int* sPrefix, long long x) {
+  int lo = 0, hi = a.B - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if ((long long)a.Hkv * sPrefix[mid] <= x) lo = mid; else hi = mid - 1;
+  }
+  SegState st;
+  st.b = lo;
+  const int nb = sPrefix[lo + 1] - sPrefix[lo];
+  const long long r = x - (long long)a.Hkv * sPrefix[lo];
+  st.hk = (int)(r / nb);
+  st.k0 = (int)(r % nb);
+  st.x = x;
+  return st;
+}
+
 template <typename T, int D, int RPW, int NTW, bool PAGED>
 __global__ void __launch_bounds__(NTW == 1 ? 288 : 160)
     decode_kernel(DecodeArgs a, int nrg) {
@@ -139,33 +187,7 @@ __global__ void __launch_bounds__(NTW == 1 ? 288 : 160)
       mbar_init(&empty[s], ncw);
     }
   }
-  {
-    // block-wide exclusive scan of chunks per sequence: sPrefix[b] = sum_{b'<b} n_b'
-    const int nthr = blockDim.x;
-    const int per = (a.B + nthr - 1) / nthr;
-    const int lo = threadIdx.x * per;
-    const int hi = min(a.B, lo + per);
-    int tsum = 0;
-    for (int b = lo; b < hi; ++b) tsum += (attended_len(a, b, blockIdx.x == 0) + kChunk - 1) / kChunk;
-    int incl = tsum;
-#pragma unroll
-    for (int m = 1; m < 32; m <<= 1) {
-      const int v = __shfl_up_sync(0xffffffffu, incl, m);
-      if (lane >= m) incl += v;
-    }
-    int* sWarpTot = reinterpret_cast<int*>(sML);  // scratch before first use of sML
-    if (lane == 31) sWarpTot[warp] = incl;
-    __syncthreads();
-    int woff = 0;
-    for (int w = 0; w < warp; ++w) woff += sWarpTot[w];
-    int run = woff + incl - tsum;
-    for (int b = lo; b < hi; ++b) {
-      sPrefix[b] = run;
-      run += (attended_len(a, b, false) + kChunk - 1) / kChunk;
-    }
-    if (hi == a.B && lo < hi) sPrefix[a.B] = run;
-    __syncthreads();
-  }
+  chunk_prefix_scan(a, sPrefix, reinterpret_cast<int*>(sML));  // sML is free until the first segment ends
   fence_barrier_init();
   fence_proxy_async_smem();
   __syncthreads();
@@ -176,21 +198,7 @@ __global__ void __launch_bounds__(NTW == 1 ? 288 : 160)
   const long long x1 = total * (blockIdx.x + 1) / a.grid;
   if (x0 >= x1) return;  // empty range: no copies issued, nothing to write
 
-  // locate the unit holding chunk x0: largest b with Hkv * prefix[b] <= x0
-  SegState st;
-  {
-    int lo = 0, hi = a.B - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if ((long long)a.Hkv * sPrefix[mid] <= x0) lo = mid; else hi = mid - 1;
-    }
-    st.b = lo;
-    const int nb = sPrefix[lo + 1] - sPrefix[lo];
-    const long long r = x0 - (long long)a.Hkv * sPrefix[lo];
-    st.hk = (int)(r / nb);
-    st.k0 = (int)(r % nb);
-    st.x = x0;
-  }
+  const SegState st = locate_chunk(a, sPrefix, x0);
 
   if (warp == ncw) {
     // ======================= producer warp ===============================
@@ -201,7 +209,25 @@ __global__ void __launch_bounds__(NTW == 1 ? 288 : 160)
       const int nb = sPrefix[p.b + 1] - sPrefix[p.b];
       const int Nb = attended_len(a, p.b, false);
       const int kend = (int)min((long long)nb, p.k0 + (x1 - p.x));
+      // page ids of the sequence, two 32-chunk windows: the second is loaded
+      // 32 chunks ahead of its use so the block-table latency stays off the issue path
+      auto page_of = [&](int ch) -> int {
+        if (ch >= kend) return -1;
+        return a.block_table[(size_t)p.b * a.max_pages_per_seq + (ch * kChunk) / a.page_size];
+      };
+      int wbase = p.k0, win0 = -1, win1 = -1;
+      if constexpr (PAGED) {
+        win0 = page_of(wbase + lane);
+        win1 = page_of(wbase + 32 + lane);
+      }
       for (int kk = p.k0; kk < kend; kk += G::STAGE_CHUNKS, ++s) {
+        if constexpr (PAGED) {
+          if (kk - wbase >= 32) {
+            wbase += 32;
+            win0 = win1;
+            win1 = page_of(wbase + 32 + lane);
+          }
+        }
         const int slot = s % G::NSTAGES;
         const uint32_t par = (uint32_t)(s / G::NSTAGES) & 1u;
         // one lane waits, the warp follows its verdict (keeps the warp converged)
@@ -226,11 +252,11 @@ __global__ void __launch_bounds__(NTW == 1 ? 288 : 160)
           // lane c < nck copies chunk c of the stage (16 tokens inside one page)
           uint32_t bytes = 0;
           size_t off = 0;
+          const int page =
+              __shfl_sync(0xffffffffu, win0, kk - wbase + min(lane, G::STAGE_CHUNKS - 1));
           if (lane < nck) {
             const int tc = t0 + lane * kChunk;
             const int ntok = min(kChunk, Nb - tc);
-            const int lp = tc / a.page_size;
-            const int page = a.block_table[(size_t)p.b * a.max_pages_per_seq + lp];
             if (page >= 0 && page < a.num_pages) {
               bytes = (uint32_t)ntok * G::TOKEN_BYTES;
               off = (((size_t)page * a.Hkv + p.hk) * a.page_size + (tc % a.page_size)) * D;

@@ -117,7 +117,8 @@ int decode_common(const kvd_params* p, const void* q, const void* k_cache, const
   a.cap_tokens = (int)(cap > INT32_MAX ? INT32_MAX : cap);
   a.qscale = p->scale * 1.4426950408889634f;  // log2(e): softmax evaluated with exp2
   a.out_bf16 = p->out_dtype == KVD_BF16;
-  a.grid = decode_grid(p->batch, p->num_kv_heads, p->max_kv_len, sms);
+  a.grid = decode_grid(p->batch, p->num_kv_heads, p->max_kv_len, sms, p->head_dim,
+                             p->dtype == KVD_BF16, (int)R);
   const cudaError_t e = launch_decode(a, p->dtype == KVD_BF16, static_cast<cudaStream_t>(stream));
   if (e == cudaErrorNotSupported) return KVD_ERR_UNSUPPORTED;
   return e == cudaSuccess ? KVD_OK : KVD_ERR_CUDA;

@@ -2,9 +2,10 @@
 //
 // Memory movement uses the bulk-copy engine (cp.async.bulk, global -> shared,
 // completion counted in bytes on an mbarrier); no cluster multicast is used
-// anywhere.  Every wait on an mbarrier is bounded: after kWaitLimit polls the
-// waiter gives up, ORs KVD_FLAG_WAIT_TIMEOUT into the status word and returns
-// false, so a broken pipeline ends the kernel instead of hanging the GPU.
+// anywhere.  Every wait on an mbarrier is bounded: after kWaitNs of wall time
+// the waiter gives up, ORs KVD_FLAG_WAIT_TIMEOUT into the status word and
+// returns false; the kernels then skip their remaining waits, so a broken
+// pipeline ends the kernel instead of hanging the GPU.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -15,9 +16,9 @@
 
 namespace kvd {
 
-// try_wait suspends the thread for a hardware-defined window per poll, so this
-// bound is on the order of a second of wall time.
-constexpr uint32_t kWaitLimit = 1u << 22;
+// A wait gives up after this much wall time (global nanosecond timer); every
+// wait in these kernels normally ends within microseconds.
+constexpr unsigned long long kWaitNs = 1000000000ull;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -52,23 +53,36 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
       : "memory");
 }
 
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+// One potentially blocking test: the thread sleeps in hardware until the phase
+// completes or about `suspend_ns` pass, so waiting warps do not take issue
+// slots from the warps doing the work.
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity,
+                                              uint32_t suspend_ns = 1000000u) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(suspend_ns)
       : "memory");
   return ok != 0;
 }
 
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
 // Bounded wait for the phase with the given parity.  Returns false (and flags
-// the status word) if the limit was reached.
+// the status word) once kWaitNs of wall time passed without completion.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status) {
-  for (uint32_t it = 0; it < kWaitLimit; ++it) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  for (;;) {
     if (mbar_try_wait(bar, parity)) return true;
+    if (global_ns() - t0 > kWaitNs) break;
   }
   if (status) atomicOr(status, KVD_FLAG_WAIT_TIMEOUT);
   return false;

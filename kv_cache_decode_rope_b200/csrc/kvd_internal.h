@@ -12,7 +12,9 @@ namespace kvd {
 
 constexpr int kChunk = 16;        // tokens per work quantum (one page of 16, or a slice of one)
 constexpr int kMaxGrid = 1024;    // upper bound on decode CTAs; sizes the workspace
-constexpr int kMaxRows = 64;      // g * q_len rows per (sequence, kv head) on the CUDA-core path
+constexpr int kMaxRows = 128;     // g * q_len rows per (sequence, kv head): tensor-core path
+constexpr int kMaxRowsCore = 64;  // ... on the CUDA-core path
+constexpr int kTcMinRows = 16;    // rows from which QK^T / PV run on the tensor cores
 constexpr int kMaxBatch = 8192;   // sequences per call (per-CTA length scan lives in shared memory)
 
 struct AppendArgs {
@@ -60,7 +62,8 @@ WorkspaceLayout workspace_layout(int B, int Hkv, int R, int D);
 cudaError_t launch_append(const AppendArgs& a, int bf16, cudaStream_t st);
 // Returns cudaErrorNotSupported when no kernel is compiled for the shape.
 cudaError_t launch_decode(const DecodeArgs& a, int bf16, cudaStream_t st);
-int decode_grid(int B, int Hkv, int max_kv_len, int num_sms);
+bool use_tensor_cores(int D, int bf16, int R);
+int decode_grid(int B, int Hkv, int max_kv_len, int num_sms, int D, int bf16, int R);
 bool decode_supported(int D, int bf16, int R);
 
 }  // namespace kvd

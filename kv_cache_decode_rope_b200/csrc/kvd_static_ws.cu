@@ -94,7 +94,8 @@ extern "C" int decode_attention_static(const kvd_params* p, const void* q, const
 
   // Carve the scratch for the grid this call launches: one partial slot per
   // (CTA, unit) pair the work split can produce, i.e. grid + units slots.
-  const int grid = decode_grid(p->batch, p->num_kv_heads, p->max_kv_len, sms);
+  const int grid = decode_grid(p->batch, p->num_kv_heads, p->max_kv_len, sms, p->head_dim,
+                             p->dtype == KVD_BF16, (int)R);
   const size_t U = (size_t)p->batch * p->num_kv_heads;
   const size_t slots = (size_t)grid + U;
   const size_t unit_off = 0;

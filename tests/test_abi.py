@@ -85,7 +85,9 @@ def test_null_params(lib):
     (dict(head_dim=256, dtype=_lib.KVD_F32), -2),    # fp32 rows of 1 KB do not fit one warp
     (dict(dtype=7), -1),
     (dict(out_dtype=3), -1),
-    (dict(num_heads=128, num_kv_heads=1), -2),      # 128 rows per unit > 64
+    (dict(num_heads=256, num_kv_heads=1), -2),      # 256 rows per unit > 128 (tensor-core path)
+    (dict(num_heads=128, num_kv_heads=1, dtype=_lib.KVD_F32), -2),  # > 64 rows on the CUDA-core path
+    (dict(num_heads=128, num_kv_heads=1, head_dim=64), -2),
     (dict(max_seq_len=0), -1),
     (dict(max_kv_len=0), -1),
     (dict(scale=float("nan")), -1),

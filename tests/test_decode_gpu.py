@@ -12,7 +12,17 @@ from kv_cache_decode_rope_b200.workloads import WORKLOADS, make_inputs
 from tests.gpu_util import (gpu_decode, gpu_step, log_error, np64, oracle_step, to_device,
                             tol_for)
 
-F32_ABS = 1e-5   # allowance for the fp32 accumulation error of a bf16-output comparison
+# fp32 error allowed on top of one bf16 ulp when comparing a bf16 output: the
+# CUDA-core path accumulates in fp32 (errors ~1e-7); the tensor-core path
+# (g * q_len >= 16, bf16, D = 128) feeds the probabilities to the MMA as bf16,
+# a relative error up to 2^-9 per weight (measured max ~5.5e-4 on these shapes).
+F32_ABS_CORE = 1e-5
+F32_ABS_TC = 1e-3
+
+
+def f32_allowance(w):
+    tc = w.dtype == "bf16" and w.head_dim == 128 and w.rows >= 16
+    return F32_ABS_TC if tc else F32_ABS_CORE
 
 pytestmark = pytest.mark.gpu
 
@@ -40,6 +50,10 @@ SHAPES = {
     "f32_d32_paged_q4": WORKLOADS["paged_cb"].with_(batch=2, dtype="f32", head_dim=32, num_heads=8,
                                                     num_kv_heads=2, len_range=(1, 150), q_len=4),
     "short_lens": WORKLOADS["paged_cb"].with_(batch=9, len_range=(1, 20)),
+    "tc_rows128": WORKLOADS["batched_gqa"].with_(batch=2, num_heads=64, num_kv_heads=2, q_len=4,
+                                                  cache_len=300),
+    "tc_rows18_paged": WORKLOADS["paged_cb"].with_(batch=3, num_heads=12, num_kv_heads=2, q_len=3,
+                                                   len_range=(1, 900)),
 }
 
 
@@ -71,7 +85,7 @@ def test_bf16_output_within_one_ulp(name):
     e = np.floor(np.log2(np.maximum(np.abs(ref_b), 1e-30)))
     err = np.abs(got - ref_b) - np.exp2(e - 7)
     log_error(f"bf16_out[{name}]", float(np.max(np.abs(got - ref_b))))
-    assert np.all(err <= F32_ABS), float(err.max())
+    assert np.all(err <= f32_allowance(w)), float(err.max())
 
 
 def test_tiny_mha_prefill_then_decode_equals_full_recompute():
