@@ -9,18 +9,23 @@
 // cache ("Flash Decoding", ferrum-sampler 0.7.0 README, Key Optimizations)
 // and merged by log-sum-exp in kernel C.
 //
-// One CTA per SM, 6 warps:
-// * warp 4 (TMA): 2-D tensor loads of 16-token K and V boxes (two 64-dim
-//   halves each, 128-byte swizzle) into a 4-stage ring of 64-token stages;
-// * warp 5 (MMA): one thread issues S = Q K^T (M = 128 query rows padded,
+// One CTA per SM, 10 warps:
+// * warp 8 (TMA): 2-D tensor loads of 16-token K and V boxes (two 64-dim
+//   halves each, 128-byte swizzle) into a ring of 64-token stages; page ids
+//   come from a prefetched window of the block table;
+// * warp 9 (MMA): one thread issues S = Q K^T (M = 64 or 128 query rows,
 //   N = 64 tokens, K = 128 dims) into a double-buffered TMEM tile, then
-//   O += P V (M = 128, N = 128 dims, K = 64 tokens) into a TMEM accumulator;
-// * warps 0-3 (softmax): thread r owns query row r: reads its S row from
-//   TMEM, masks, keeps a running max that is only raised when it grows by
-//   more than 2^8 (the accumulator is rescaled in TMEM only then), writes its
-//   probabilities as bf16 into a swizzled shared tile for the PV product, and
-//   at a unit boundary reads its O row back and writes the output or a
-//   normalised partial (o, lse).
+//   O_h += P_h V_h for the two token halves h of the stage into two TMEM
+//   accumulators; P is passed as bf16 high part + bf16 residual (two passes
+//   over V), which keeps the probabilities to ~16 significant bits;
+// * warps 0-7 (softmax): warpgroup h (warps 4h .. 4h+3) owns tokens
+//   32h .. 32h+31 of every stage; thread (warp, lane) owns one query row of
+//   the unit (rows spread over the four TMEM sub-partitions).  It reads its S
+//   row from TMEM, masks, keeps a reference max raised only when the running
+//   max grows by more than 2^8 (then its O row is rescaled in TMEM), and
+//   writes its probabilities into a swizzled shared tile for the PV product.
+//   At a unit boundary the two halves are merged by log-sum-exp and the
+//   output (or a normalised partial) is written.
 // The work split over units and CTAs is the one of the CUDA-core kernel, so
 // the same merge kernel finishes split units.
 #include <cuda.h>
@@ -36,79 +41,86 @@ namespace {
 
 constexpr int TC_D = 128;
 constexpr int TC_STAGE = 64;                      // tokens per stage
+constexpr int TC_HALF = TC_STAGE / 2;             // tokens per softmax warpgroup
 constexpr int TC_CHUNKS = TC_STAGE / kChunk;      // 16-token boxes per stage
-constexpr int TC_NS = 4;                          // ring depth
-constexpr int TC_ROWS = 128;                      // MMA M (query rows, padded)
-constexpr int TC_THREADS = 192;
-constexpr uint32_t TC_TMEM_COLS = 256;            // S0 | S1 | O
+constexpr int TC_THREADS = 320;                   // 8 softmax warps + TMA + MMA
+constexpr int TC_SOFTMAX_THREADS = 256;
+constexpr int WARP_TMA = 8, WARP_MMA = 9;
+constexpr uint32_t TC_TMEM_COLS = 512;            // S0 | S1 | O_0 | O_1
 constexpr uint32_t COL_S = 0, COL_O = 128;
 constexpr float kRescaleThreshold = 8.0f;         // log2 units
 
+// M = MMA rows (query rows of a unit, padded): 64 or 128.
+template <int M>
 struct TcSmem {
-  static constexpr int HALF_Q = TC_ROWS * 128;        // 16 KB: 128 rows x 64 dims
+  static constexpr int NS = M == 128 ? 3 : 4;          // ring depth (shared memory bound)
+  static constexpr int HALF_Q = M * 128;               // M rows x 64 dims
   static constexpr int Q = 0;                          // 2 halves
   static constexpr int KV = Q + 2 * HALF_Q;            // ring
   static constexpr int K_HALF = TC_STAGE * 128;        // 8 KB: 64 tokens x 64 dims
   static constexpr int STAGE = 4 * K_HALF;             // K (2 halves) + V (2 halves)
-  static constexpr int P = KV + TC_NS * STAGE;         // 2 x [128 rows x 64 tokens]
-  static constexpr int P_BUF = TC_ROWS * 128;
-  static constexpr int BAR = P + 2 * P_BUF;
-  static constexpr int NBAR = 2 * TC_NS + 10;
+  static constexpr int P = KV + NS * STAGE;            // 2 buffers x (hi, lo) x [M rows x 64 tokens]
+  static constexpr int P_BUF = M * 128;
+  static constexpr int BAR = P + 4 * P_BUF;
+  static constexpr int NBAR = 2 * NS + 10;
   static constexpr int TMEM_SLOT = BAR + NBAR * 8;
-  static constexpr int SCRATCH = TMEM_SLOT + 16;       // 8 ints for the scan
-  static constexpr int PREFIX = SCRATCH + 32;
+  static constexpr int ML = TMEM_SLOT + 16;            // [2][M] x (m, l) for the epilogue merge
+  static constexpr int SCRATCH = ML + 2 * M * 8;       // one int per warp for the scan
+  static constexpr int PREFIX = SCRATCH + 64;
   static size_t bytes(int B) { return (size_t)PREFIX + (size_t)(B + 1) * 4 + 1024; }
 };
 
-template <bool PAGED>
+template <bool PAGED, int M>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmk,
                      const __grid_constant__ CUtensorMap tmv) {
+  using S = TcSmem<M>;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  unsigned char* sQ = smem + TcSmem::Q;
-  unsigned char* sKV = smem + TcSmem::KV;
-  unsigned char* sP = smem + TcSmem::P;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + TcSmem::BAR);
-  uint64_t* full = bars;                  // TMA -> MMA (+ softmax on tail stages)
-  uint64_t* empty = bars + TC_NS;         // PV done -> TMA
-  uint64_t* s_full = bars + 2 * TC_NS;    // QK done -> softmax
+  unsigned char* sQ = smem + S::Q;
+  unsigned char* sKV = smem + S::KV;
+  unsigned char* sP = smem + S::P;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::BAR);
+  uint64_t* full = bars;                  // TMA -> MMA (+ softmax on short stages)
+  uint64_t* empty = bars + S::NS;         // PV done -> TMA
+  uint64_t* s_full = bars + 2 * S::NS;    // QK done -> softmax
   uint64_t* s_free = s_full + 2;          // S read -> MMA
   uint64_t* p_full = s_free + 2;          // P written -> MMA
   uint64_t* p_free = p_full + 2;          // PV done -> softmax
   uint64_t* q_full = p_free + 2;          // Q written -> MMA
   uint64_t* mma_done = q_full + 1;        // all issued MMAs complete (exit)
-  uint32_t* sTmem = reinterpret_cast<uint32_t*>(smem + TcSmem::TMEM_SLOT);
-  int* sScratch = reinterpret_cast<int*>(smem + TcSmem::SCRATCH);
-  int* sPrefix = reinterpret_cast<int*>(smem + TcSmem::PREFIX);
+  uint32_t* sTmem = reinterpret_cast<uint32_t*>(smem + S::TMEM_SLOT);
+  float2* sML = reinterpret_cast<float2*>(smem + S::ML);
+  int* sScratch = reinterpret_cast<int*>(smem + S::SCRATCH);
+  int* sPrefix = reinterpret_cast<int*>(smem + S::PREFIX);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
   {  // stale ring contents must be finite: start from zeros
     uint4* z = reinterpret_cast<uint4*>(sKV);
-    for (int k = threadIdx.x; k < TC_NS * TcSmem::STAGE / 16; k += blockDim.x)
+    for (int k = threadIdx.x; k < S::NS * S::STAGE / 16; k += blockDim.x)
       z[k] = make_uint4(0, 0, 0, 0);
   }
   if (threadIdx.x == 0) {
-    for (int s = 0; s < TC_NS; ++s) {
+    for (int s = 0; s < S::NS; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&s_full[b], 1);
-      mbar_init(&s_free[b], 4);
-      mbar_init(&p_full[b], 4);
+      mbar_init(&s_free[b], 8);
+      mbar_init(&p_full[b], 8);
       mbar_init(&p_free[b], 1);
     }
-    mbar_init(q_full, 4);
+    mbar_init(q_full, 8);
     mbar_init(mma_done, 1);
   }
-  if (warp == 5) {
+  if (warp == WARP_MMA) {
     tmem_alloc(sTmem, TC_TMEM_COLS);
     tmem_relinquish();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == WARP_TMA && lane == 0) {
     prefetch_tensormap(&tmk);
     prefetch_tensormap(&tmv);
   }
@@ -127,7 +139,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 
   if (x0 < x1) {
     const SegState st = locate_chunk(a, sPrefix, x0);
-    if (warp == 4) {
+    if (warp == WARP_TMA) {
       // ============================ TMA warp ===============================
       int g = 0;
       bool failed = false;
@@ -152,9 +164,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             win0 = win1;
             win1 = page_of(c.b, wbase + 32 + lane, kend);
           }
-          const int slot = g % TC_NS;
+          const int slot = g % S::NS;
           int ok = 1;
-          if (lane == 0) ok = mbar_wait(&empty[slot], ((uint32_t)(g / TC_NS) & 1u) ^ 1u, a.status);
+          if (lane == 0) ok = mbar_wait(&empty[slot], ((uint32_t)(g / S::NS) & 1u) ^ 1u, a.status);
           ok = __shfl_sync(0xffffffffu, ok, 0);
           if (!ok) { failed = true; break; }
           const int nck = min(TC_CHUNKS, kend - kk);
@@ -177,12 +189,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           if (lane == 0) mbar_arrive_expect_tx(&full[slot], bytes);
           __syncwarp();
           if (row >= 0) {
-            unsigned char* dk = sKV + slot * TcSmem::STAGE + lane * kChunk * 128;
-            unsigned char* dv = dk + 2 * TcSmem::K_HALF;
+            unsigned char* dk = sKV + slot * S::STAGE + lane * kChunk * 128;
+            unsigned char* dv = dk + 2 * S::K_HALF;
             tma_load_2d(dk, &tmk, 0, row, &full[slot]);
-            tma_load_2d(dk + TcSmem::K_HALF, &tmk, 64, row, &full[slot]);
+            tma_load_2d(dk + S::K_HALF, &tmk, 64, row, &full[slot]);
             tma_load_2d(dv, &tmv, 0, row, &full[slot]);
-            tma_load_2d(dv + TcSmem::K_HALF, &tmv, 64, row, &full[slot]);
+            tma_load_2d(dv + S::K_HALF, &tmv, 64, row, &full[slot]);
           }
           __syncwarp();
         }
@@ -191,32 +203,34 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         if (++c.hk == a.Hkv) { c.hk = 0; ++c.b; }
       }
       if (lane == 0) {  // every issued copy lands before the CTA may exit
-        for (int k = max(0, g - TC_NS); k < g; ++k)
-          if (!mbar_wait(&full[k % TC_NS], (uint32_t)(k / TC_NS) & 1u, a.status)) break;
+        for (int k = max(0, g - S::NS); k < g; ++k)
+          if (!mbar_wait(&full[k % S::NS], (uint32_t)(k / S::NS) & 1u, a.status)) break;
       }
-    } else if (warp == 5) {
+    } else if (warp == WARP_MMA) {
       // ============================ MMA warp ===============================
       if (lane == 0) {
-        constexpr uint32_t idesc_qk = idesc_bf16_f32(TC_ROWS, TC_STAGE, false);
-        constexpr uint32_t idesc_pv = idesc_bf16_f32(TC_ROWS, TC_D, true);
-        const uint32_t q_addr = smem_u32(sQ);
-        const uint32_t kv_addr = smem_u32(sKV);
-        const uint32_t p_addr = smem_u32(sP);
+        constexpr uint32_t idesc_qk = idesc_bf16_f32(M, TC_STAGE, false);
+        constexpr uint32_t idesc_pv = idesc_bf16_f32(M, TC_D, true);
+        // descriptors of the tile bases; a byte offset b inside a tile adds b >> 4
+        const uint64_t dq = sw128_desc(smem_u32(sQ), 16, 1024);
+        const uint64_t dkv = sw128_desc(smem_u32(sKV), 16, 1024);
+        const uint64_t dp = sw128_desc(smem_u32(sP), 16, 1024);
+        const uint64_t dv = sw128_desc(smem_u32(sKV), S::K_HALF, 1024);
         int g = 0, seg = 0;
         bool failed = false;
         // S = Q K^T for global stage gg into S buffer gg % 2
         auto issue_qk = [&](int gg) -> bool {
-          const int slot = gg % TC_NS;
-          if (!mbar_wait(&full[slot], (uint32_t)(gg / TC_NS) & 1u, a.status)) return false;
+          const int slot = gg % S::NS;
+          if (!mbar_wait(&full[slot], (uint32_t)(gg / S::NS) & 1u, a.status)) return false;
           if (!mbar_wait(&s_free[gg & 1], ((uint32_t)(gg >> 1) & 1u) ^ 1u, a.status)) return false;
           tc_fence_after();
-          const uint32_t k_addr = kv_addr + slot * TcSmem::STAGE;
+          const uint32_t kofs = (uint32_t)slot * S::STAGE;
 #pragma unroll
           for (int ks = 0; ks < TC_D / 16; ++ks) {
             const uint32_t off = (uint32_t)(ks & 3) * 32u;  // 16 dims = 32 bytes inside the row
-            const uint64_t ad = sw128_desc(q_addr + (ks >> 2) * TcSmem::HALF_Q + off, 16, 1024);
-            const uint64_t bd = sw128_desc(k_addr + (ks >> 2) * TcSmem::K_HALF + off, 16, 1024);
-            tc_mma_bf16(tmem + COL_S + (uint32_t)(gg & 1) * TC_STAGE, ad, bd, idesc_qk, ks > 0);
+            tc_mma_bf16(tmem + COL_S + (uint32_t)(gg & 1) * TC_STAGE,
+                        dq + (((ks >> 2) * S::HALF_Q + off) >> 4),
+                        dkv + ((kofs + (ks >> 2) * S::K_HALF + off) >> 4), idesc_qk, ks > 0);
           }
           tc_commit(&s_full[gg & 1]);
           return true;
@@ -234,15 +248,20 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             if (k + 1 < n && !issue_qk(gg + 1)) { failed = true; break; }
             if (!mbar_wait(&p_full[gg & 1], (uint32_t)(gg >> 1) & 1u, a.status)) { failed = true; break; }
             tc_fence_after();
-            const uint32_t v_addr = kv_addr + (gg % TC_NS) * TcSmem::STAGE + 2 * TcSmem::K_HALF;
-            const uint32_t pb = p_addr + (uint32_t)(gg & 1) * TcSmem::P_BUF;
+            const uint32_t vofs = (uint32_t)(gg % S::NS) * S::STAGE + 2 * S::K_HALF;
+            // token half h of the stage goes to accumulator O_h; P = P_hi + P_lo
 #pragma unroll
-            for (int ks = 0; ks < TC_STAGE / 16; ++ks) {
-              const uint64_t ad = sw128_desc(pb + ks * 32u, 16, 1024);
-              const uint64_t bd = sw128_desc(v_addr + ks * 2048u, TcSmem::K_HALF, 1024);
-              tc_mma_bf16(tmem + COL_O, ad, bd, idesc_pv, (k > 0 || ks > 0) ? 1u : 0u);
-            }
-            tc_commit(&empty[gg % TC_NS]);
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+              for (int part = 0; part < 2; ++part) {
+                const uint32_t pofs = (uint32_t)((gg & 1) * 2 + part) * S::P_BUF;
+#pragma unroll
+                for (int ks = 2 * h; ks < 2 * h + 2; ++ks)
+                  tc_mma_bf16(tmem + COL_O + (uint32_t)h * TC_D, dp + ((pofs + ks * 32u) >> 4),
+                              dv + ((vofs + ks * 2048u) >> 4), idesc_pv,
+                              (k > 0 || part > 0 || ks > 2 * h) ? 1u : 0u);
+              }
+            tc_commit(&empty[gg % S::NS]);
             tc_commit(&p_free[gg & 1]);
           }
           g += n;
@@ -257,15 +276,23 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       }
       __syncwarp();
     } else {
-      // ========================= softmax warps 0-3 =========================
-      // Tile row (= TMEM lane) p = 32 * warp + lane holds query row qr = 4 * lane + warp,
-      // so the real rows of a small group spread over all four warps / schedulers.
-      const int p = warp * 32 + lane;
-      const int qr = 4 * lane + warp;
-      const uint32_t t_lane = tmem + ((uint32_t)(warp * 32) << 16);
-      const bool row_ok = qr < a.R;
-      const bool warp_rows = warp < a.R;                    // any real row in this warp
-      const int di = row_ok ? qr / a.g : 0;                 // new-token index of the row
+      // ========================= softmax warps 0-7 =========================
+      // Sub-partition sp = warp % 4 reaches TMEM lanes 32 sp .. 32 sp + 31.
+      // M = 128: lane l there is tile row 32 sp + l; M = 64: lanes 0-15 hold
+      // tile rows 16 sp + l.  Tile row p holds query row qr = 4 l + sp, so the
+      // real rows of a small group spread over all four sub-partitions.
+      constexpr int RPT = M / 4;                            // tile rows per sub-partition
+      const int sp = warp & 3;
+      const int hw = warp >> 2;                              // token half of the stage
+      const bool lane_row = lane < RPT;
+      const int p = sp * RPT + lane;                         // tile row (if lane_row)
+      const int qr = 4 * lane + sp;
+      const int tid = threadIdx.x;                           // 0 .. 255
+      const uint32_t t_lane = tmem + ((uint32_t)(sp * 32) << 16);
+      const uint32_t col_o = COL_O + (uint32_t)hw * TC_D;
+      const bool row_ok = lane_row && qr < a.R;
+      const bool warp_rows = sp < a.R;                       // any real row in this warp
+      const int di = row_ok ? qr / a.g : 0;                  // new-token index of the row
       int g = 0, seg = 0;
       bool failed = false;
       SegState c = st;
@@ -276,20 +303,18 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         const int kend = (int)min((long long)nb, c.k0 + (x1 - c.x));
         const int n = (kend - c.k0 + TC_CHUNKS - 1) / TC_CHUNKS;
         const int u = c.b * a.Hkv + c.hk;
-        const int vis = row_ok ? Lb + di + 1 : 0;           // visible tokens of this row
+        const int vis = row_ok ? Lb + di + 1 : 0;            // visible tokens of this row
 
-        // -- query row qr into tile row p of the swizzled K-major tile (zeros for padding)
-        {
+        // -- query row qr, dims 64 hw .. 64 hw + 63, into tile row p (zeros for padding)
+        if (lane_row) {
           const int h = c.hk * a.g + (row_ok ? qr % a.g : 0);
           const uint4* src = reinterpret_cast<const uint4*>(
               reinterpret_cast<const __nv_bfloat16*>(a.q) + (((size_t)c.b * a.T + di) * a.Hq + h) * TC_D);
 #pragma unroll
-          for (int hh = 0; hh < 2; ++hh)
-#pragma unroll
-            for (int ch = 0; ch < 8; ++ch) {
-              const uint4 v = row_ok ? src[hh * 8 + ch] : make_uint4(0, 0, 0, 0);
-              *reinterpret_cast<uint4*>(sQ + hh * TcSmem::HALF_Q + p * 128 + ((ch ^ (p & 7)) << 4)) = v;
-            }
+          for (int ch = 0; ch < 8; ++ch) {
+            const uint4 v = row_ok ? src[hw * 8 + ch] : make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4*>(sQ + hw * S::HALF_Q + p * 128 + ((ch ^ (p & 7)) << 4)) = v;
+          }
         }
         fence_proxy_async_smem();
         __syncwarp();
@@ -298,23 +323,19 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         float m = -INFINITY, l = 0.f;
         for (int k = 0; k < n; ++k) {
           const int gg = g + k;
-          const int slot = gg % TC_NS;
+          const int slot = gg % S::NS;
           const int t0 = (c.k0 + k * TC_CHUNKS) * kChunk;
           const int nvalid = min(min(TC_CHUNKS, kend - c.k0 - k * TC_CHUNKS) * kChunk, Nb - t0);
           const bool tail = (nvalid < TC_STAGE) || (t0 + TC_STAGE > Lb + 1);
           if (!failed && !mbar_wait(&s_full[gg & 1], (uint32_t)(gg >> 1) & 1u, a.status)) failed = true;
           tc_fence_after();
-          float x[TC_STAGE];
+          float x[TC_HALF];
           {
-            uint32_t s0[32], s1[32];
-            tmem_ld32(t_lane + COL_S + (uint32_t)(gg & 1) * TC_STAGE, s0);
-            tmem_ld32(t_lane + COL_S + (uint32_t)(gg & 1) * TC_STAGE + 32, s1);
+            uint32_t sr[32];
+            tmem_ld32(t_lane + COL_S + (uint32_t)(gg & 1) * TC_STAGE + hw * TC_HALF, sr);
             tmem_ld_wait();
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              x[j] = __uint_as_float(s0[j]) * a.qscale;
-              x[j + 32] = __uint_as_float(s1[j]) * a.qscale;
-            }
+            for (int j = 0; j < TC_HALF; ++j) x[j] = __uint_as_float(sr[j]) * a.qscale;
           }
           tc_fence_before();
           __syncwarp();
@@ -322,8 +343,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 
           float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-          for (int j = 0; j < TC_STAGE; ++j) {
-            if (!row_ok || (tail && (j >= nvalid || t0 + j >= vis))) x[j] = -INFINITY;
+          for (int j = 0; j < TC_HALF; ++j) {
+            const int tj = hw * TC_HALF + j;                 // token of the stage
+            if (!row_ok || (tail && (tj >= nvalid || t0 + tj >= vis))) x[j] = -INFINITY;
             mx4[j & 3] = fmaxf(mx4[j & 3], x[j]);
           }
           const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
@@ -337,55 +359,62 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             m = mx;
             l *= alpha;
           }
-          uint32_t pk[TC_STAGE / 2];
+          uint32_t pk[TC_HALF / 2], pl[TC_HALF / 2];   // bf16 pairs: high part, residual
           if (warp_rows) {
             float ps4[4] = {0.f, 0.f, 0.f, 0.f};
             const float mref = (m == -INFINITY) ? 0.f : m;
 #pragma unroll
-            for (int j = 0; j < TC_STAGE; j += 2) {
+            for (int j = 0; j < TC_HALF; j += 2) {
               const float p0 = fast_exp2(x[j] - mref), p1 = fast_exp2(x[j + 1] - mref);
               ps4[(j >> 1) & 3] += p0 + p1;
-              pk[j / 2] = pack_bf16x2(p0, p1);
+              const uint32_t hi = pack_bf16x2(p0, p1);
+              pk[j / 2] = hi;
+              pl[j / 2] = pack_bf16x2(p0 - __uint_as_float(hi << 16), p1 - __uint_as_float(hi & 0xffff0000u));
             }
             l += (ps4[0] + ps4[1]) + (ps4[2] + ps4[3]);
           } else {
 #pragma unroll
-            for (int j = 0; j < TC_STAGE / 2; ++j) pk[j] = 0u;
+            for (int j = 0; j < TC_HALF / 2; ++j) { pk[j] = 0u; pl[j] = 0u; }
           }
 
           // P buffer (gg & 1) is free once PV(gg - 2) completed
           if (!failed && !mbar_wait(&p_free[gg & 1], ((uint32_t)(gg >> 1) & 1u) ^ 1u, a.status)) failed = true;
           if (__any_sync(0xffffffffu, rescale)) {
-            // O must hold PV(gg - 1) before it is scaled in place
+            // O_hw must hold PV(gg - 1) before it is scaled in place
             if (!failed && !mbar_wait(&p_free[(gg - 1) & 1], (uint32_t)((gg - 1) >> 1) & 1u, a.status))
               failed = true;
             tc_fence_after();
 #pragma unroll
             for (int cb = 0; cb < TC_D / 32; ++cb) {
               uint32_t o[32];
-              tmem_ld32(t_lane + COL_O + cb * 32, o);
+              tmem_ld32(t_lane + col_o + cb * 32, o);
               tmem_ld_wait();
 #pragma unroll
               for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-              tmem_st32(t_lane + COL_O + cb * 32, o);
+              tmem_st32(t_lane + col_o + cb * 32, o);
             }
             tmem_st_wait();
           }
-          {
-            unsigned char* prow = sP + (gg & 1) * TcSmem::P_BUF + p * 128;
+          if (lane_row) {
+            // tokens 32 hw .. 32 hw + 31 = 16-byte chunks 4 hw .. 4 hw + 3 of the row
+            unsigned char* prow = sP + ((gg & 1) * 2) * S::P_BUF + p * 128;
 #pragma unroll
-            for (int ch = 0; ch < 8; ++ch)
-              *reinterpret_cast<uint4*>(prow + ((ch ^ (p & 7)) << 4)) =
+            for (int ch = 0; ch < 4; ++ch) {
+              const int cc = hw * 4 + ch;
+              *reinterpret_cast<uint4*>(prow + ((cc ^ (p & 7)) << 4)) =
                   make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+              *reinterpret_cast<uint4*>(prow + S::P_BUF + ((cc ^ (p & 7)) << 4)) =
+                  make_uint4(pl[4 * ch], pl[4 * ch + 1], pl[4 * ch + 2], pl[4 * ch + 3]);
+            }
           }
           if (nvalid < TC_STAGE) {
             // rows past the valid tokens hold whatever the cache held there: zero them in V
-            if (!failed && !mbar_wait(&full[slot], (uint32_t)(gg / TC_NS) & 1u, a.status)) failed = true;
-            unsigned char* vbase = sKV + slot * TcSmem::STAGE + 2 * TcSmem::K_HALF;
+            if (!failed && !mbar_wait(&full[slot], (uint32_t)(gg / S::NS) & 1u, a.status)) failed = true;
+            unsigned char* vbase = sKV + slot * S::STAGE + 2 * S::K_HALF;
             const int nz = (TC_STAGE - nvalid) * 8;  // 16-byte pieces per half
-            for (int e = p; e < 2 * nz; e += 128) {
+            for (int e = tid; e < 2 * nz; e += TC_SOFTMAX_THREADS) {
               const int hh = e / nz, q = e % nz;
-              *reinterpret_cast<uint4*>(vbase + hh * TcSmem::K_HALF + nvalid * 128 + q * 16) =
+              *reinterpret_cast<uint4*>(vbase + hh * S::K_HALF + nvalid * 128 + q * 16) =
                   make_uint4(0, 0, 0, 0);
             }
           }
@@ -395,56 +424,67 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           if (lane == 0) mbar_arrive(&p_full[gg & 1]);
         }
 
-        // -- unit segment done: O row out
+        // -- unit segment done: merge the two token halves, write the row
         const int gl = g + n - 1;
         if (!failed && !mbar_wait(&p_free[gl & 1], (uint32_t)(gl >> 1) & 1u, a.status)) failed = true;
         tc_fence_after();
+        if (lane_row) sML[hw * M + p] = make_float2(m, l);
+        named_bar_sync(1, TC_SOFTMAX_THREADS);
+        float2 mo = make_float2(-INFINITY, 0.f);
+        if (lane_row) mo = sML[(1 - hw) * M + p];
+        const float m0 = hw == 0 ? m : mo.x, l0 = hw == 0 ? l : mo.y;
+        const float m1 = hw == 0 ? mo.x : m, l1 = hw == 0 ? mo.y : l;
+        const float mm = fmaxf(m0, m1);
+        const float ms = (mm == -INFINITY) ? 0.f : mm;
+        const float w0 = fast_exp2(m0 - ms), w1 = fast_exp2(m1 - ms);
+        const float L = w0 * l0 + w1 * l1;
+        const float inv = (L > 0.f) ? 1.f / L : 0.f;
+        const float s0 = w0 * inv, s1 = w1 * inv;
         const bool whole = (c.k0 == 0) && (kend == nb);
-        const float inv = (l > 0.f) ? 1.f / l : 0.f;
         const long long slot_idx = (long long)blockIdx.x + u;
         const int h = c.hk * a.g + (row_ok ? qr % a.g : 0);
+        // warpgroup hw writes dims 64 hw .. 64 hw + 63 of the row
 #pragma unroll
-        for (int cb = 0; cb < TC_D / 32; ++cb) {
-          uint32_t o[32];
-          tmem_ld32(t_lane + COL_O + cb * 32, o);
+        for (int cb = 0; cb < 2; ++cb) {
+          const int d0 = hw * 64 + cb * 32;
+          uint32_t o0[32], o1[32];
+          tmem_ld32(t_lane + COL_O + d0, o0);
+          tmem_ld32(t_lane + COL_O + TC_D + d0, o1);
           tmem_ld_wait();
+          float ov[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) ov[j] = __uint_as_float(o0[j]) * s0 + __uint_as_float(o1[j]) * s1;
           if (row_ok) {
             if (whole) {
-              const size_t ob = (((size_t)c.b * a.T + di) * a.Hq + h) * TC_D + cb * 32;
+              const size_t ob = (((size_t)c.b * a.T + di) * a.Hq + h) * TC_D + d0;
               if (a.out_bf16) {
                 uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + ob);
 #pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                  uint32_t w[4];
-#pragma unroll
-                  for (int e = 0; e < 4; ++e)
-                    w[e] = pack_bf16x2(__uint_as_float(o[q4 * 8 + 2 * e]) * inv,
-                                       __uint_as_float(o[q4 * 8 + 2 * e + 1]) * inv);
-                  dst[q4] = make_uint4(w[0], w[1], w[2], w[3]);
-                }
+                for (int q4 = 0; q4 < 4; ++q4)
+                  dst[q4] = make_uint4(pack_bf16x2(ov[8 * q4], ov[8 * q4 + 1]), pack_bf16x2(ov[8 * q4 + 2], ov[8 * q4 + 3]),
+                                       pack_bf16x2(ov[8 * q4 + 4], ov[8 * q4 + 5]), pack_bf16x2(ov[8 * q4 + 6], ov[8 * q4 + 7]));
               } else {
                 float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(a.out) + ob);
 #pragma unroll
                 for (int q4 = 0; q4 < 8; ++q4)
-                  dst[q4] = make_float4(__uint_as_float(o[4 * q4]) * inv, __uint_as_float(o[4 * q4 + 1]) * inv,
-                                        __uint_as_float(o[4 * q4 + 2]) * inv, __uint_as_float(o[4 * q4 + 3]) * inv);
+                  dst[q4] = make_float4(ov[4 * q4], ov[4 * q4 + 1], ov[4 * q4 + 2], ov[4 * q4 + 3]);
               }
             } else {
-              float4* dst = reinterpret_cast<float4*>(a.part_o + ((size_t)slot_idx * a.R + qr) * TC_D + cb * 32);
+              float4* dst = reinterpret_cast<float4*>(a.part_o + ((size_t)slot_idx * a.R + qr) * TC_D + d0);
 #pragma unroll
               for (int q4 = 0; q4 < 8; ++q4)
-                dst[q4] = make_float4(__uint_as_float(o[4 * q4]) * inv, __uint_as_float(o[4 * q4 + 1]) * inv,
-                                      __uint_as_float(o[4 * q4 + 2]) * inv, __uint_as_float(o[4 * q4 + 3]) * inv);
+                dst[q4] = make_float4(ov[4 * q4], ov[4 * q4 + 1], ov[4 * q4 + 2], ov[4 * q4 + 3]);
             }
           }
         }
-        if (row_ok && !whole)
-          a.part_lse[(size_t)slot_idx * a.R + qr] = (l > 0.f) ? m + fast_log2(l) : -INFINITY;
+        if (row_ok && !whole && hw == 0)
+          a.part_lse[(size_t)slot_idx * a.R + qr] = (L > 0.f) ? ms + fast_log2(L) : -INFINITY;
         if (threadIdx.x == 0) {
           if (c.k0 == 0) a.unit_ctas[u].x = blockIdx.x;
           if (kend == nb) a.unit_ctas[u].y = blockIdx.x;
         }
         tc_fence_before();  // the O reads above precede the next segment's first PV
+        named_bar_sync(1, TC_SOFTMAX_THREADS);   // sML is reused by the next segment
 
         g += n;
         ++seg;
@@ -457,7 +497,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 5) tmem_dealloc(tmem, TC_TMEM_COLS);
+  if (warp == WARP_MMA) tmem_dealloc(tmem, TC_TMEM_COLS);
 }
 
 // ---------------------------------------------------------------- host side
@@ -490,7 +530,7 @@ bool make_map(CUtensorMap* map, const void* base, unsigned long long rows) {
   return r == CUDA_SUCCESS;
 }
 
-template <bool PAGED>
+template <bool PAGED, int M>
 cudaError_t launch_tc(const DecodeArgs& a, cudaStream_t st) {
   const unsigned long long rows =
       PAGED ? (unsigned long long)a.num_pages * a.Hkv * a.page_size
@@ -498,7 +538,7 @@ cudaError_t launch_tc(const DecodeArgs& a, cudaStream_t st) {
   if (rows >= (1ull << 31)) return cudaErrorNotSupported;  // TMA row coordinate is int32
   CUtensorMap mk, mv;
   if (!make_map(&mk, a.k_cache, rows) || !make_map(&mv, a.v_cache, rows)) return cudaErrorNotSupported;
-  const size_t smem = TcSmem::bytes(a.B);
+  const size_t smem = TcSmem<M>::bytes(a.B);
   if (smem > 227 * 1024) return cudaErrorNotSupported;
   static std::atomic<unsigned long long> attr_done{0};
   int dev = 0;
@@ -506,12 +546,12 @@ cudaError_t launch_tc(const DecodeArgs& a, cudaStream_t st) {
   if (e != cudaSuccess) return e;
   const unsigned long long bit = 1ull << (dev & 63);
   if (!(attr_done.load() & bit)) {
-    e = cudaFuncSetAttribute(decode_tc_kernel<PAGED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(decode_tc_kernel<PAGED, M>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              227 * 1024);
     if (e != cudaSuccess) return e;
     attr_done.fetch_or(bit);
   }
-  decode_tc_kernel<PAGED><<<a.grid, TC_THREADS, smem, st>>>(a, mk, mv);
+  decode_tc_kernel<PAGED, M><<<a.grid, TC_THREADS, smem, st>>>(a, mk, mv);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const long long warps = (long long)a.B * a.Hkv * a.R;
@@ -522,7 +562,8 @@ cudaError_t launch_tc(const DecodeArgs& a, cudaStream_t st) {
 }  // namespace
 
 cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t st) {
-  return a.block_table ? launch_tc<true>(a, st) : launch_tc<false>(a, st);
+  if (a.R <= 64) return a.block_table ? launch_tc<true, 64>(a, st) : launch_tc<false, 64>(a, st);
+  return a.block_table ? launch_tc<true, 128>(a, st) : launch_tc<false, 128>(a, st);
 }
 
 }  // namespace kvd
