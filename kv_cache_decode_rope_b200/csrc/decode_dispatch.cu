@@ -34,7 +34,12 @@ int decode_grid(int B, int Hkv, int max_kv_len, int num_sms, int D, int bf16, in
 }
 
 cudaError_t launch_decode(const DecodeArgs& a, int bf16, cudaStream_t st) {
-  if (use_tensor_cores(a.D, bf16, a.R)) return launch_decode_tc(a, st);
+  if (use_tensor_cores(a.D, bf16, a.R)) {
+    const cudaError_t e = launch_decode_tc(a, st);
+    // very large batches do not fit the tensor-core kernel's shared memory:
+    // units of up to 64 rows then run on the CUDA-core kernel
+    if (e != cudaErrorNotSupported || a.R > kMaxRowsCore) return e;
+  }
   if (a.block_table)
     return bf16 ? launch_decode_bf16_paged(a, st) : launch_decode_f32_paged(a, st);
   return bf16 ? launch_decode_bf16_contig(a, st) : launch_decode_f32_contig(a, st);
