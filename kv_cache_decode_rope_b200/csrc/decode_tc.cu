@@ -379,6 +379,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         p_lo = p_hi + C::P_TILE;
       }
       const int pch0 = (tok0 % 64) / 8;                      // first 16-byte chunk in the row
+      // Scores enter the exponent as fma(q . k, qs, -m) with qs > 0.  A
+      // negative scale flips the sign of q instead (exact in bf16), so the
+      // maximum of the raw products stays the maximum of the scaled scores; a
+      // zero scale becomes a tiny one, which gives the same all-ones weights
+      // while keeping -inf * qs = -inf for masked tokens.
+      const uint32_t qflip = a.qscale < 0.f ? 0x80008000u : 0u;
+      const float qs = fmaxf(fabsf(a.qscale), 1e-30f);
       int g = 0;
       bool failed = false;
       SegState c = st;
@@ -401,7 +408,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 #pragma unroll
           for (int k8 = 0; k8 < NCH; ++k8) {
             const int ch = cs * 4 + k8;
-            const uint4 v = row_ok ? src[hw * 8 + ch] : make_uint4(0, 0, 0, 0);
+            uint4 v = row_ok ? src[hw * 8 + ch] : make_uint4(0, 0, 0, 0);
+            v.x ^= qflip; v.y ^= qflip; v.z ^= qflip; v.w ^= qflip;
             *reinterpret_cast<uint4*>(sQ + hw * C::HALF_Q + p * 128 + ((ch ^ (p & 7)) << 4)) = v;
           }
         }
@@ -417,29 +425,41 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           const bool tail = (nvalid < ST) || (t0 + ST > Lb + 1);
           if (!failed && !mbar_wait(&s_full[gg & 1], (uint32_t)(gg >> 1) & 1u, a.status)) failed = true;
           tc_fence_after();
-          float x[32];
+          uint32_t sr[32];   // raw scores q . k of this thread's 32 tokens
           {
-            uint32_t sr[32];
             const uint32_t sa = t_lane + C::COL_S + (uint32_t)(gg & 1) * ST + hw * HALF;
             if constexpr (C::STACK) tmem_ld16x2_32(sa, sr);
             else tmem_ld32(sa, sr);
             tmem_ld_wait();
-#pragma unroll
-            for (int j = 0; j < 32; ++j) x[j] = __uint_as_float(sr[j]) * a.qscale;
           }
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&s_free[gg & 1]);
 
-          float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+          // Masking only on the stages that hold a causal edge, the end of the
+          // cache or a partial chunk (the same for every thread).  Outside them
+          // padding rows keep their finite scores: a padding row only feeds its
+          // own O row, which is never written out.
+          if (tail) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int tj = tok0 + j;                         // token of the stage
-            if (!row_ok || (tail && (tj >= nvalid || t0 + tj >= vis))) x[j] = -INFINITY;
-            mx4[j & 3] = fmaxf(mx4[j & 3], x[j]);
+            for (int j = 0; j < 32; ++j) {
+              const int tj = tok0 + j;                       // token of the stage
+              if (!row_ok || tj >= nvalid || t0 + tj >= vis) sr[j] = __float_as_uint(-INFINITY);
+            }
           }
-          float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+          float mx;
+          {
+            float t16[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) t16[j] = fmaxf(__uint_as_float(sr[j]), __uint_as_float(sr[j + 16]));
+#pragma unroll
+            for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+              for (int j = 0; j < w; ++j) t16[j] = fmaxf(t16[j], t16[j + w]);
+            mx = t16[0];
+          }
           if constexpr (C::STACK) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+          mx *= qs;                                          // qs > 0: the scaled maximum
           float alpha = 1.f;
           bool rescale = false;
           if (mx > m + kRescaleThreshold) {   // raise the reference max only on a large jump
@@ -452,18 +472,22 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           }
           uint32_t pk[16], pl[16];   // bf16 pairs: high part (top 16 bits), residual (top 16 bits)
           if (warp_rows) {
-            float ps4[4] = {0.f, 0.f, 0.f, 0.f};
             const float mref = (m == -INFINITY) ? 0.f : m;
+            const float2 qs2 = make_float2(qs, qs), nm2 = make_float2(-mref, -mref);
+            float2 sum2 = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int j = 0; j < 32; j += 2) {
-              const float p0 = fast_exp2(x[j] - mref), p1 = fast_exp2(x[j + 1] - mref);
-              ps4[(j >> 1) & 3] += p0 + p1;
-              const uint32_t b0 = __float_as_uint(p0), b1 = __float_as_uint(p1);
-              pk[j / 2] = hi16x2(b0, b1);
-              pl[j / 2] = hi16x2(__float_as_uint(p0 - __uint_as_float(b0 & 0xffff0000u)),
-                                 __float_as_uint(p1 - __uint_as_float(b1 & 0xffff0000u)));
+            for (int j = 0; j < 16; ++j) {
+              const float2 e = __ffma2_rn(make_float2(__uint_as_float(sr[2 * j]), __uint_as_float(sr[2 * j + 1])),
+                                          qs2, nm2);
+              const float2 pp = make_float2(fast_exp2(e.x), fast_exp2(e.y));
+              sum2 = __fadd2_rn(sum2, pp);
+              const uint32_t b0 = __float_as_uint(pp.x), b1 = __float_as_uint(pp.y);
+              const float2 hi = make_float2(__uint_as_float(b0 & 0xffff0000u), __uint_as_float(b1 & 0xffff0000u));
+              const float2 lo = __ffma2_rn(hi, make_float2(-1.f, -1.f), pp);   // exact: pp - hi
+              pk[j] = hi16x2(b0, b1);
+              pl[j] = hi16x2(__float_as_uint(lo.x), __float_as_uint(lo.y));
             }
-            l += (ps4[0] + ps4[1]) + (ps4[2] + ps4[3]);
+            l += sum2.x + sum2.y;
           } else {
 #pragma unroll
             for (int j = 0; j < 16; ++j) { pk[j] = 0u; pl[j] = 0u; }
