@@ -67,7 +67,7 @@ struct TcCfg {
   static constexpr int CH = ST / kChunk;               // 16-token boxes per stage
   static constexpr int HALF = ST / 2;                  // tokens per softmax warpgroup
   static constexpr int NK = STACK ? 3 : 4;             // K ring depth
-  static constexpr int NV = STACK ? 2 : 4;             // V ring depth
+  static constexpr int NV = STACK ? 3 : 4;             // V ring depth
   static constexpr int HALF_Q = MQ * 128;              // MQ rows x 64 dims
   static constexpr int DHALF = ST * 128;               // one 64-dim half of a K or V stage
   static constexpr int KVSTAGE = 2 * DHALF;
@@ -75,12 +75,11 @@ struct TcCfg {
   static constexpr int KR = Q + 2 * HALF_Q;            // K ring
   static constexpr int VR = KR + NK * KVSTAGE;         // V ring
   static constexpr int P = VR + NV * KVSTAGE;
-  // P tile(s), 128 rows x 128 bytes each:
-  //  STACK: one per token half h; row 32 s + r holds the high part of tile
-  //         row 16 s + r, row 32 s + 16 + r its residual.
-  //  else:  [high, residual]; token half h in bytes [64 h, 64 h + 64) of a row.
+  // P: with STACK it lives in tensor memory (the columns of the S buffer it
+  // was computed from); otherwise two 128-row x 128-byte shared tiles [high,
+  // residual], token half h in bytes [64 h, 64 h + 64) of a row.
   static constexpr int P_TILE = 128 * 128;
-  static constexpr int BAR = P + 2 * P_TILE;
+  static constexpr int BAR = P + (STACK ? 0 : 2 * P_TILE);
   static constexpr int NBAR = 2 * NK + 2 * NV + 2 + 2 + 2 + 2 + 1 + 2;
   static constexpr int TMEM_SLOT = BAR + NBAR * 8;
   static constexpr int ML = TMEM_SLOT + 16;            // [2 halves][MQ] (m, l) for the merge
@@ -181,7 +180,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   uint64_t* v_full = k_empty + NK;        // V loader -> PV issuer (+ softmax on short stages)
   uint64_t* v_empty = v_full + NV;        // PV done -> V loader
   uint64_t* s_full = v_empty + NV;        // QK done -> softmax            [S buffer]
-  uint64_t* s_free = s_full + 2;          // S read -> QK issuer           [S buffer]
+  uint64_t* s_free = s_full + 2;          // S buffer reusable -> QK issuer [S buffer]
   uint64_t* p_full = s_free + 2;          // P half written -> PV issuer   [token half]
   uint64_t* p_free = p_full + 2;          // PV of a half done -> softmax  [token half]
   uint64_t* q_full = p_free + 2;          // Q written -> QK issuer
@@ -210,7 +209,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&s_full[b], 1);
-      mbar_init(&s_free[b], 8);
+      // STACK: P overwrites S in tensor memory, so the buffer is free once the
+      // PV product of its stage is done (one commit); otherwise once the 8
+      // softmax warps have read S
+      mbar_init(&s_free[b], C::STACK ? 1 : 8);
       mbar_init(&p_full[b], 4);
       mbar_init(&p_free[b], 1);
       mbar_init(&mma_done[b], 1);
@@ -311,13 +313,14 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
               if (!mbar_wait(&p_full[h], (uint32_t)gg & 1u, a.status)) { failed = true; break; }
               tc_fence_after();
               if constexpr (C::STACK) {
-                // rows [high; residual] of P_h against the 64 tokens of half h
+                // rows [high; residual] of P_h (tensor memory, 32 columns of S
+                // buffer gg % 2 from column 64 h) against the 64 tokens of half h
 #pragma unroll
                 for (int ks = 0; ks < HALF / 16; ++ks) {
                   const int t = h * HALF + ks * 16;
-                  tc_mma_bf16(tmem + C::COL_O + (uint32_t)h * TC_D,
-                              dp + (((uint32_t)h * C::P_TILE + ks * 32) >> 4),
-                              dv + ((vofs + t * 128) >> 4), idesc_pv, (k > 0 || ks > 0) ? 1u : 0u);
+                  tc_mma_bf16_ta(tmem + C::COL_O + (uint32_t)h * TC_D,
+                                 tmem + C::COL_S + (uint32_t)(gg & 1) * ST + (uint32_t)(h * 64 + ks * 8),
+                                 dv + ((vofs + t * 128) >> 4), idesc_pv, (k > 0 || ks > 0) ? 1u : 0u);
                 }
               } else {
 #pragma unroll
@@ -334,6 +337,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
               tc_commit(&p_free[h]);
             }
             tc_commit(&v_empty[slot]);
+            if constexpr (C::STACK) tc_commit(&s_free[gg & 1]);   // P(gg) read: the S buffer is free
           }
           g += n;
           c.x += kend - c.k0;
@@ -368,54 +372,62 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       const bool row_ok = qr < a.R;
       const bool warp_rows = sp < a.R;                       // any real row in this warp
       const int di = row_ok ? qr / a.g : 0;                  // new-token index of the row
-      // this thread's slice of the P tile(s): row and byte offset of its 32 tokens
-      unsigned char* p_hi;
-      unsigned char* p_lo;
-      if constexpr (C::STACK) {
-        p_hi = sP + hw * C::P_TILE + (32 * sp + rl) * 128;
-        p_lo = p_hi + 16 * 128;
-      } else {
-        p_hi = sP + p * 128;
-        p_lo = p_hi + C::P_TILE;
-      }
-      const int pch0 = (tok0 % 64) / 8;                      // first 16-byte chunk in the row
-      // Scores enter the exponent as fma(q . k, qs, -m) with qs > 0.  A
-      // negative scale flips the sign of q instead (exact in bf16), so the
-      // maximum of the raw products stays the maximum of the scaled scores; a
-      // zero scale becomes a tiny one, which gives the same all-ones weights
-      // while keeping -inf * qs = -inf for masked tokens.
-      const uint32_t qflip = a.qscale < 0.f ? 0x80008000u : 0u;
-      const float qs = fmaxf(fabsf(a.qscale), 1e-30f);
+      // MQ = 128: this thread's row of the shared P tiles and its first 16-byte
+      // chunk there (MQ = 64 keeps P in tensor memory)
+      unsigned char* p_hi = sP + p * 128;
+      unsigned char* p_lo = p_hi + C::P_TILE;
+      const int pch0 = (tok0 % 64) / 8;
+      // Scores enter the exponent as fma(q . k, qs, -m).  With qs > 0 the
+      // reference comes from the largest raw product, with qs < 0 from the
+      // smallest; masked tokens take the raw value that the scale maps to -inf.
+      // A zero scale becomes a tiny positive one: the same all-ones weights,
+      // while masked tokens still map to -inf.
+      const bool qneg = a.qscale < 0.f;
+      const float qs = qneg ? a.qscale : fmaxf(a.qscale, 1e-30f);
+      const uint32_t mask_raw = __float_as_uint(qneg ? INFINITY : -INFINITY);
+      // q rows of unit (b, hk) into the Q tile: tile row p, dim half hw, 16-byte
+      // chunks 4 cs .. 4 cs + 3 (pairs) or all 8; padding rows read as zeros
+      auto issue_q = [&](int b, int hk) {
+        const int h = hk * a.g + (row_ok ? qr % a.g : 0);
+        const uint4* src = reinterpret_cast<const uint4*>(
+            reinterpret_cast<const __nv_bfloat16*>(a.q) + (((size_t)b * a.T + di) * a.Hq + h) * TC_D);
+        constexpr int NCH = C::STACK ? 4 : 8;
+#pragma unroll
+        for (int k8 = 0; k8 < NCH; ++k8) {
+          const int ch = cs * 4 + k8;
+          cp_async16(sQ + hw * C::HALF_Q + p * 128 + ((ch ^ (p & 7)) << 4), src + hw * 8 + ch,
+                     row_ok ? 16u : 0u);
+        }
+      };
+      // the copies have landed: hand the tile to the QK issuer
+      auto publish_q = [&]() {
+        cp_async_wait_all();
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(q_full);
+      };
+      issue_q(st.b, st.hk);
+      publish_q();
+      int Nb_cur = attended_len(a, st.b, false);
       int g = 0;
       bool failed = false;
       SegState c = st;
       while (c.x < x1) {
         const int nb = sPrefix[c.b + 1] - sPrefix[c.b];
-        const int Nb = attended_len(a, c.b, false);
+        const int Nb = Nb_cur;
         const int Lb = Nb - a.T;
         const int kend = (int)min((long long)nb, c.k0 + (x1 - c.x));
         const int n = (kend - c.k0 + CH - 1) / CH;
         const int u = c.b * a.Hkv + c.hk;
         const int vis = row_ok ? Lb + di + 1 : 0;            // visible tokens of this row
 
-        // -- query row qr into tile row p (zeros for padding rows): dim half hw,
-        //    chunks 4 cs .. 4 cs + 3 (pairs) or all 8
-        {
-          const int h = c.hk * a.g + (row_ok ? qr % a.g : 0);
-          const uint4* src = reinterpret_cast<const uint4*>(
-              reinterpret_cast<const __nv_bfloat16*>(a.q) + (((size_t)c.b * a.T + di) * a.Hq + h) * TC_D);
-          constexpr int NCH = C::STACK ? 4 : 8;
-#pragma unroll
-          for (int k8 = 0; k8 < NCH; ++k8) {
-            const int ch = cs * 4 + k8;
-            uint4 v = row_ok ? src[hw * 8 + ch] : make_uint4(0, 0, 0, 0);
-            v.x ^= qflip; v.y ^= qflip; v.z ^= qflip; v.w ^= qflip;
-            *reinterpret_cast<uint4*>(sQ + hw * C::HALF_Q + p * 128 + ((ch ^ (p & 7)) << 4)) = v;
-          }
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(q_full);
+        // the next unit of this CTA's range, whose q is fetched during the last
+        // stage of this one (the Q tile is free once that stage's QK is done)
+        const bool has_next = c.x + (kend - c.k0) < x1;
+        const int nx_hk = (c.hk + 1 == a.Hkv) ? 0 : c.hk + 1;
+        const int nx_b = (c.hk + 1 == a.Hkv) ? c.b + 1 : c.b;
+        // length of the next unit's sequence, loaded now and used after this unit
+        if (has_next && nx_b != c.b) Nb_cur = attended_len(a, nx_b, false);
 
         float m = -INFINITY, l = 0.f;
         for (int k = 0; k < n; ++k) {
@@ -425,6 +437,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           const bool tail = (nvalid < ST) || (t0 + ST > Lb + 1);
           if (!failed && !mbar_wait(&s_full[gg & 1], (uint32_t)(gg >> 1) & 1u, a.status)) failed = true;
           tc_fence_after();
+          const bool last = k == n - 1;
+          if (last && has_next) issue_q(nx_b, nx_hk);
           uint32_t sr[32];   // raw scores q . k of this thread's 32 tokens
           {
             const uint32_t sa = t_lane + C::COL_S + (uint32_t)(gg & 1) * ST + hw * HALF;
@@ -434,7 +448,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           }
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&s_free[gg & 1]);
+          if constexpr (!C::STACK) {
+            if (lane == 0) mbar_arrive(&s_free[gg & 1]);
+          }
 
           // Masking only on the stages that hold a causal edge, the end of the
           // cache or a partial chunk (the same for every thread).  Outside them
@@ -444,22 +460,34 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
               const int tj = tok0 + j;                       // token of the stage
-              if (!row_ok || tj >= nvalid || t0 + tj >= vis) sr[j] = __float_as_uint(-INFINITY);
+              if (!row_ok || tj >= nvalid || t0 + tj >= vis) sr[j] = mask_raw;
             }
           }
-          float mx;
+          float mx;   // raw product that the scale maps to the largest score
           {
             float t16[16];
+            if (!qneg) {
 #pragma unroll
-            for (int j = 0; j < 16; ++j) t16[j] = fmaxf(__uint_as_float(sr[j]), __uint_as_float(sr[j + 16]));
+              for (int j = 0; j < 16; ++j) t16[j] = fmaxf(__uint_as_float(sr[j]), __uint_as_float(sr[j + 16]));
 #pragma unroll
-            for (int w = 8; w >= 1; w >>= 1)
+              for (int w = 8; w >= 1; w >>= 1)
 #pragma unroll
-              for (int j = 0; j < w; ++j) t16[j] = fmaxf(t16[j], t16[j + w]);
+                for (int j = 0; j < w; ++j) t16[j] = fmaxf(t16[j], t16[j + w]);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 16; ++j) t16[j] = fminf(__uint_as_float(sr[j]), __uint_as_float(sr[j + 16]));
+#pragma unroll
+              for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+                for (int j = 0; j < w; ++j) t16[j] = fminf(t16[j], t16[j + w]);
+            }
             mx = t16[0];
           }
-          if constexpr (C::STACK) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-          mx *= qs;                                          // qs > 0: the scaled maximum
+          if constexpr (C::STACK) {
+            const float o = __shfl_xor_sync(0xffffffffu, mx, 16);
+            mx = qneg ? fminf(mx, o) : fmaxf(mx, o);
+          }
+          mx *= qs;                                          // the largest scaled score
           float alpha = 1.f;
           bool rescale = false;
           if (mx > m + kRescaleThreshold) {   // raise the reference max only on a large jump
@@ -493,10 +521,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             for (int j = 0; j < 16; ++j) { pk[j] = 0u; pl[j] = 0u; }
           }
 
-          // the P tile of half hw is free, and O_hw holds every earlier stage,
-          // once PV(gg - 1) of this half completed
+          // PV(gg - 1) of this half completed: O_hw holds every earlier stage,
+          // the shared P tile (MQ = 128) is free, and the PV issuer has taken
+          // phase gg - 1 of p_full[hw], so this stage's arrival cannot run two
+          // phases ahead of its wait
           if (!failed && !mbar_wait(&p_free[hw], (uint32_t)(gg - 1) & 1u, a.status)) failed = true;
-          if (__any_sync(0xffffffffu, rescale)) {
+          const bool any_rescale = __any_sync(0xffffffffu, rescale);
+          if (any_rescale) {
             tc_fence_after();
 #pragma unroll
             for (int cb = 0; cb < TC_D; cb += 16) {
@@ -509,13 +540,29 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             }
             tmem_st_wait();
           }
+          if constexpr (C::STACK) {
+            // P_hw into tensor memory over the S values just read: thread cs = 0
+            // writes the high row (lane 32 sp + rl), cs = 1 the residual row
+            // (lane 32 sp + 16 + rl), each over all 64 tokens of the half, so
+            // the pair trades the 32 tokens of the part the other one writes
+            uint32_t pr[32];
 #pragma unroll
-          for (int ch = 0; ch < 4; ++ch) {
-            const int sw = ((pch0 + ch) ^ (rl & 7)) << 4;
-            *reinterpret_cast<uint4*>(p_hi + sw) =
-                make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
-            *reinterpret_cast<uint4*>(p_lo + sw) =
-                make_uint4(pl[4 * ch], pl[4 * ch + 1], pl[4 * ch + 2], pl[4 * ch + 3]);
+            for (int j = 0; j < 16; ++j) {
+              const uint32_t got = __shfl_xor_sync(0xffffffffu, cs ? pk[j] : pl[j], 16);
+              pr[j] = cs ? got : pk[j];          // tokens 2j, 2j + 1
+              pr[16 + j] = cs ? pl[j] : got;     // tokens 32 + 2j, 33 + 2j
+            }
+            tmem_st32(t_lane + C::COL_S + (uint32_t)(gg & 1) * ST + (uint32_t)hw * 64, pr);
+            tmem_st_wait();
+          } else {
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) {
+              const int sw = ((pch0 + ch) ^ (rl & 7)) << 4;
+              *reinterpret_cast<uint4*>(p_hi + sw) =
+                  make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+              *reinterpret_cast<uint4*>(p_lo + sw) =
+                  make_uint4(pl[4 * ch], pl[4 * ch + 1], pl[4 * ch + 2], pl[4 * ch + 3]);
+            }
           }
           if (nvalid < ST) {
             // V rows past the valid tokens hold whatever the cache (or an older
@@ -536,6 +583,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&p_full[hw]);
+          if (last && has_next) publish_q();
         }
 
         // -- unit segment done: merge the two token halves, write the row
