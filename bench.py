@@ -238,11 +238,14 @@ def run_ours(args, rank, world, local):
         decode(q, seq)
     torch.cuda.synchronize()
 
-    # The timed loop replays the step's two library calls from CUDA graphs
+    # The timed loop replays the step's two library calls from a CUDA graph
     # captured through the same public API: the kernels, their arguments and
     # the work are those of the eager calls, but the host enqueues a step in a
-    # few microseconds, so the device never idles waiting for Python and the
-    # events time the kernels alone.  --launch eager times the plain calls.
+    # few microseconds, so the device never idles waiting for Python, and the
+    # kernels' programmatic dependent launch overlaps each kernel's set-up with
+    # the tail of the one before.  Two more loops replay the decode call and
+    # the append call alone to time them separately (the per-kernel figures).
+    # --launch eager times plain calls instead.
     if args.launch == "graph":
         side = torch.cuda.Stream(device=dev)
         side.wait_stream(torch.cuda.current_stream())
@@ -251,15 +254,18 @@ def run_ours(args, rank, world, local):
             decode(q, seq)
         torch.cuda.current_stream().wait_stream(side)
         torch.cuda.synchronize()
-        g_app, g_dec = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        g_step, g_app, g_dec = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_step):
+            append(q, kn, vn, seq)
+            decode(q, seq)
         with torch.cuda.graph(g_app):
             append(q, kn, vn, seq)
         with torch.cuda.graph(g_dec):
             decode(q, seq)
         torch.cuda.synchronize()
-        run_append = g_app.replay
-        run_decode = g_dec.replay
+        run_step, run_append, run_decode = g_step.replay, g_app.replay, g_dec.replay
         for _ in range(3):
+            run_step()
             run_append()
             run_decode()
         torch.cuda.synchronize()
@@ -270,8 +276,29 @@ def run_ours(args, rank, world, local):
         def run_decode():
             decode(q, seq)
 
+        def run_step():
+            run_append()
+            run_decode()
+
+    def timed(fn, n, before=None):
+        """Per-iteration device times (ms) of n calls of fn, each after an
+        untimed call of `before` (the rest of the step), L2 flushed before each
+        call when the inputs fit in it."""
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(n)]
+        for e0, e1 in evs:
+            if before is not None:
+                before()
+            if flush:
+                flush_buf.add_(1)
+            e0.record()
+            fn()
+            e1.record()
+        torch.cuda.synchronize()
+        return [e0.elapsed_time(e1) for e0, e1 in evs]
+
     K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
@@ -283,18 +310,18 @@ def run_ours(args, rank, world, local):
             if flush:
                 flush_buf.add_(1)
             ev[k][0].record()
-            run_append()
+            run_step()
             ev[k][1].record()
-            run_decode()
-            ev[k][2].record()
         t_all1.record()
         torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
-    step_ms = [ev[k][0].elapsed_time(ev[k][2]) for k in range(K)]
-    dec_ms = [ev[k][1].elapsed_time(ev[k][2]) for k in range(K)]
-    app_ms = [ev[k][0].elapsed_time(ev[k][1]) for k in range(K)]
+    step_ms = [e0.elapsed_time(e1) for e0, e1 in ev]
     total_ms = sum(step_ms) if flush else t_all0.elapsed_time(t_all1)
+    # per-kernel figures, outside the timed region
+    Kk = min(K, 200)
+    dec_ms = timed(run_decode, Kk, before=run_append)
+    app_ms = timed(run_append, Kk, before=run_decode)
     if status.item() != 0:
         raise RuntimeError(f"device status flags set during the bench: {status.item()}")
 
@@ -344,8 +371,8 @@ def run_ours(args, rank, world, local):
     e2e_ms = e0.elapsed_time(e1) / Ke
 
     res = dict(total_ms=total_ms, step_ms=statistics.median(step_ms),
-               mean_step_ms=total_ms / K, dec_ms=sum(dec_ms) / K, dec_med=statistics.median(dec_ms),
-               app_ms=sum(app_ms) / K, e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, bytes=nbytes,
+               mean_step_ms=total_ms / K, dec_ms=sum(dec_ms) / len(dec_ms), dec_med=statistics.median(dec_ms),
+               app_ms=sum(app_ms) / len(app_ms), e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, bytes=nbytes,
                clocks=clk.summary(), flush=flush, cache_bytes=cache_bytes, w=w, mkl=mkl)
     return res
 

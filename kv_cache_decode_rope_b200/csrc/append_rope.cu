@@ -17,6 +17,7 @@
 
 #include "kvd_device.cuh"
 #include "kvd_internal.h"
+#include "kvd_launch.h"
 
 namespace kvd {
 namespace {
@@ -45,6 +46,7 @@ __global__ void __launch_bounds__(256) append_rope_kernel(AppendArgs a) {
   __shared__ double s_cos[HALF];
   __shared__ double s_sin[HALF];
 
+  grid_dep_launch();
   const int b = blockIdx.x / a.T;
   const int i = blockIdx.x % a.T;
   const long long pos = (long long)a.seq_lens[b] + i;
@@ -56,6 +58,9 @@ __global__ void __launch_bounds__(256) append_rope_kernel(AppendArgs a) {
     s_cos[j] = c;
     s_sin[j] = s;
   }
+  // everything above read only seq_lens: wait for the previous kernel before
+  // touching q, k/v, the caches or the status word
+  grid_dep_wait();
 
   // Where position `pos` of sequence b lives; -1 if it is outside the cache.
   long long slot_base = -1;  // element offset of (kv head 0, pos); heads are `head_stride` apart
@@ -137,14 +142,13 @@ cudaError_t launch_t(const AppendArgs& a, cudaStream_t st) {
   int threads = 32;
   while (threads < 256 && threads < work / (16 / (int)sizeof(T))) threads *= 2;
   switch (a.D) {
-    case 16: append_rope_kernel<T, 16><<<grid, threads, 0, st>>>(a); break;
-    case 32: append_rope_kernel<T, 32><<<grid, threads, 0, st>>>(a); break;
-    case 64: append_rope_kernel<T, 64><<<grid, threads, 0, st>>>(a); break;
-    case 128: append_rope_kernel<T, 128><<<grid, threads, 0, st>>>(a); break;
-    case 256: append_rope_kernel<T, 256><<<grid, threads, 0, st>>>(a); break;
+    case 16: return launch_pdl(append_rope_kernel<T, 16>, dim3(grid), dim3(threads), 0, st, a);
+    case 32: return launch_pdl(append_rope_kernel<T, 32>, dim3(grid), dim3(threads), 0, st, a);
+    case 64: return launch_pdl(append_rope_kernel<T, 64>, dim3(grid), dim3(threads), 0, st, a);
+    case 128: return launch_pdl(append_rope_kernel<T, 128>, dim3(grid), dim3(threads), 0, st, a);
+    case 256: return launch_pdl(append_rope_kernel<T, 256>, dim3(grid), dim3(threads), 0, st, a);
     default: return cudaErrorNotSupported;
   }
-  return cudaGetLastError();
 }
 
 }  // namespace

@@ -33,13 +33,23 @@ int decode_grid(int B, int Hkv, int max_kv_len, int num_sms, int D, int bf16, in
   return (int)g;
 }
 
-cudaError_t launch_decode(const DecodeArgs& a, int bf16, cudaStream_t st) {
+// Virtual chunks charged per unit in the work split (the cost of a unit
+// boundary, in 16-token chunks of streaming): about two 128-token stages for
+// the tensor-core kernel (epilogue, pipeline refill), half that for the
+// CUDA-core kernel, whose CTAs each stream at half an SM's bandwidth.
+constexpr int kSegCostTc = 16;
+constexpr int kSegCostCore = 8;
+
+cudaError_t launch_decode(const DecodeArgs& args, int bf16, cudaStream_t st) {
+  DecodeArgs a = args;
   if (use_tensor_cores(a.D, bf16, a.R)) {
+    a.seg_cost = kSegCostTc;
     const cudaError_t e = launch_decode_tc(a, st);
     // very large batches do not fit the tensor-core kernel's shared memory:
     // units of up to 64 rows then run on the CUDA-core kernel
     if (e != cudaErrorNotSupported || a.R > kMaxRowsCore) return e;
   }
+  a.seg_cost = kSegCostCore;
   if (a.block_table)
     return bf16 ? launch_decode_bf16_paged(a, st) : launch_decode_f32_paged(a, st);
   return bf16 ? launch_decode_bf16_contig(a, st) : launch_decode_f32_contig(a, st);

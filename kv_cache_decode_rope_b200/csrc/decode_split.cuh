@@ -37,6 +37,7 @@
 
 #include "kvd_device.cuh"
 #include "kvd_internal.h"
+#include "kvd_launch.h"
 
 namespace kvd {
 namespace {
@@ -96,8 +97,15 @@ __device__ __forceinline__ int attended_len(const DecodeArgs& a, int b, bool fla
   return (int)N;
 }
 
-// Block-wide exclusive scan of chunks per sequence: sPrefix[b] = sum over
-// b' < b of ceil(N_b' / 16), sPrefix[B] = total.  All threads of the block
+// The work split.  Each unit (sequence b, kv head) occupies seg_cost virtual
+// chunks followed by its ceil(N_b / 16) real chunks in one index space, units
+// in order (b, then kv head); CTA c takes the slice [total c / grid,
+// total (c + 1) / grid).  The virtual chunks charge every unit boundary a
+// fixed cost, so a CTA whose slice crosses many short units gets fewer real
+// chunks.  Virtual chunks are never loaded.
+//
+// Block-wide exclusive scan of weighted chunks per sequence: sPrefix[b] = sum
+// over b' < b of (ceil(N_b' / 16) + seg_cost), sPrefix[B] = total.  All threads of the block
 // call it; `scratch` holds one int per warp.  Ends with __syncthreads.
 __device__ __forceinline__ void chunk_prefix_scan(const DecodeArgs& a, int* sPrefix, int* scratch) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -106,7 +114,8 @@ __device__ __forceinline__ void chunk_prefix_scan(const DecodeArgs& a, int* sPre
   const int lo = threadIdx.x * per;
   const int hi = min(a.B, lo + per);
   int tsum = 0;
-  for (int b = lo; b < hi; ++b) tsum += (attended_len(a, b, blockIdx.x == 0) + kChunk - 1) / kChunk;
+  for (int b = lo; b < hi; ++b)
+    tsum += (attended_len(a, b, blockIdx.x == 0) + kChunk - 1) / kChunk + a.seg_cost;
   int incl = tsum;
 #pragma unroll
   for (int m = 1; m < 32; m <<= 1) {
@@ -120,13 +129,13 @@ __device__ __forceinline__ void chunk_prefix_scan(const DecodeArgs& a, int* sPre
   int run = woff + incl - tsum;
   for (int b = lo; b < hi; ++b) {
     sPrefix[b] = run;
-    run += (attended_len(a, b, false) + kChunk - 1) / kChunk;
+    run += (attended_len(a, b, false) + kChunk - 1) / kChunk + a.seg_cost;
   }
   if (hi == a.B && lo < hi) sPrefix[a.B] = run;
   __syncthreads();
 }
 
-// The unit (sequence b, kv head hk) and chunk within it of global chunk x:
+// The unit (sequence b, kv head hk) and weighted chunk within it of global index x:
 // largest b with Hkv * prefix[b] <= x, then the head and chunk inside b.
 __device__ __forceinline__ SegState locate_chunk(const DecodeArgs& a, const int* sPrefix, long long x) {
   int lo = 0, hi = a.B - 1;
@@ -142,6 +151,36 @@ __device__ __forceinline__ SegState locate_chunk(const DecodeArgs& a, const int*
   st.k0 = (int)(r % nb);
   st.x = x;
   return st;
+}
+
+// A CTA's share of the unit at `c` (slice ending at x1): real chunks
+// [k0, kend) of the unit's nb; empty when kend <= k0 (the slice ends inside
+// the unit's virtual chunks).
+struct Seg {
+  int nb, k0, kend;
+  long long next_x;  // weighted index where the next unit's share starts
+  __device__ bool empty() const { return kend <= k0; }
+  __device__ bool whole() const { return k0 == 0 && kend == nb; }
+};
+__device__ __forceinline__ Seg seg_of(const DecodeArgs& a, const int* sPrefix, const SegState& c,
+                                      long long x1) {
+  const int ext = sPrefix[c.b + 1] - sPrefix[c.b];
+  const int kend_ext = (int)min((long long)ext, c.k0 + (x1 - c.x));
+  Seg s;
+  s.nb = ext - a.seg_cost;
+  s.k0 = max(c.k0 - a.seg_cost, 0);
+  s.kend = kend_ext - a.seg_cost;
+  s.next_x = c.x + (kend_ext - c.k0);
+  return s;
+}
+__device__ __forceinline__ void next_unit(const DecodeArgs& a, SegState& c, const Seg& s) {
+  c.x = s.next_x;
+  c.k0 = 0;
+  if (++c.hk == a.Hkv) { c.hk = 0; ++c.b; }
+}
+// Does the slice reach real chunks of the unit after the one ending at next_x?
+__device__ __forceinline__ bool next_has_work(const DecodeArgs& a, const Seg& s, long long x1) {
+  return x1 - s.next_x > a.seg_cost;
 }
 
 template <typename T, int D, int RPW, int NTW, bool PAGED>
@@ -191,6 +230,8 @@ __global__ void __launch_bounds__(NTW == 1 ? 288 : 160)
   fence_barrier_init();
   fence_proxy_async_smem();
   __syncthreads();
+  grid_dep_wait();      // q, the caches and the workspace are ready
+  grid_dep_launch();
 
   const long long total = (long long)a.Hkv * sPrefix[a.B];
   if (blockIdx.x == 0 && threadIdx.x == 0) *a.total_chunks = total;
@@ -205,22 +246,23 @@ __global__ void __launch_bounds__(NTW == 1 ? 288 : 160)
     int s = 0;
     bool failed = false;
     SegState p = st;
-    while (p.x < x1 && !failed) {
-      const int nb = sPrefix[p.b + 1] - sPrefix[p.b];
+    for (; p.x < x1 && !failed; next_unit(a, p, seg_of(a, sPrefix, p, x1))) {
+      const Seg sg = seg_of(a, sPrefix, p, x1);
+      if (sg.empty()) continue;
       const int Nb = attended_len(a, p.b, false);
-      const int kend = (int)min((long long)nb, p.k0 + (x1 - p.x));
+      const int kend = sg.kend;
       // page ids of the sequence, two 32-chunk windows: the second is loaded
       // 32 chunks ahead of its use so the block-table latency stays off the issue path
       auto page_of = [&](int ch) -> int {
         if (ch >= kend) return -1;
         return a.block_table[(size_t)p.b * a.max_pages_per_seq + (ch * kChunk) / a.page_size];
       };
-      int wbase = p.k0, win0 = -1, win1 = -1;
+      int wbase = sg.k0, win0 = -1, win1 = -1;
       if constexpr (PAGED) {
         win0 = page_of(wbase + lane);
         win1 = page_of(wbase + 32 + lane);
       }
-      for (int kk = p.k0; kk < kend; kk += G::STAGE_CHUNKS, ++s) {
+      for (int kk = sg.k0; kk < kend; kk += G::STAGE_CHUNKS, ++s) {
         if constexpr (PAGED) {
           if (kk - wbase >= 32) {
             wbase += 32;
@@ -278,9 +320,6 @@ __global__ void __launch_bounds__(NTW == 1 ? 288 : 160)
         }
         __syncwarp();
       }
-      p.x += kend - p.k0;
-      p.k0 = 0;
-      if (++p.hk == a.Hkv) { p.hk = 0; ++p.b; }
     }
     // drain: every issued copy lands before the CTA may exit
     if (lane == 0) {
@@ -308,11 +347,12 @@ __global__ void __launch_bounds__(NTW == 1 ? 288 : 160)
   int s = 0;
   bool failed = false;
   SegState c = st;
-  while (c.x < x1) {
-    const int nb = sPrefix[c.b + 1] - sPrefix[c.b];
+  for (; c.x < x1; next_unit(a, c, seg_of(a, sPrefix, c, x1))) {
+    const Seg sg = seg_of(a, sPrefix, c, x1);
+    if (sg.empty()) continue;
     const int Nb = attended_len(a, c.b, false);
     const int Lb = Nb - a.T;  // first new-token position (may be <= 0 after clamping)
-    const int kend = (int)min((long long)nb, c.k0 + (x1 - c.x));
+    const int kend = sg.kend;
     const int u = c.b * a.Hkv + c.hk;
 
     // -- segment init: q rows of this warp, pre-scaled for exp2
@@ -345,7 +385,7 @@ __global__ void __launch_bounds__(NTW == 1 ? 288 : 160)
       vis_own[i] = (rglob < a.R) ? Lb + rglob / a.g + 1 : Nb;
     }
 
-    for (int kk = c.k0; kk < kend; kk += G::STAGE_CHUNKS, ++s) {
+    for (int kk = sg.k0; kk < kend; kk += G::STAGE_CHUNKS, ++s) {
       const int slot = s % G::NSTAGES;
       const uint32_t par = (uint32_t)(s / G::NSTAGES) & 1u;
       if (!failed && !mbar_wait(&full[slot], par, a.status)) failed = true;
@@ -516,7 +556,7 @@ __global__ void __launch_bounds__(NTW == 1 ? 288 : 160)
     }
     named_bar_sync(1, ncons);
 
-    const bool whole = (c.k0 == 0) && (kend == nb);
+    const bool whole = sg.whole();
     const long long slot_idx = (long long)blockIdx.x + u;
     for (int e = threadIdx.x; e < nrg * RPW * D; e += ncons) {
       const int rgi = e / (RPW * D);
@@ -547,22 +587,24 @@ __global__ void __launch_bounds__(NTW == 1 ? 288 : 160)
       }
     }
     if (threadIdx.x == 0) {
-      if (c.k0 == 0) a.unit_ctas[u].x = blockIdx.x;
-      if (kend == nb) a.unit_ctas[u].y = blockIdx.x;
+      if (sg.k0 == 0) a.unit_ctas[u].x = blockIdx.x;
+      if (sg.kend == sg.nb) a.unit_ctas[u].y = blockIdx.x;
     }
     named_bar_sync(1, ncons);
-
-    c.x += kend - c.k0;
-    c.k0 = 0;
-    if (++c.hk == a.Hkv) { c.hk = 0; ++c.b; }
   }
 }
 
 // Kernel C: one warp per (unit, row) merges the partials of units split over
 // several CTAs: out = sum_s 2^(lse_s - LSE) o_s with LSE = log2 sum_s 2^lse_s.
+// Lane j fetches the log-sum-exp of partials j, j + 32, ...; each lane then
+// reads its D / 32 dimensions of four partial rows at a time, so the merge
+// costs a handful of dependent memory round trips whatever the split count.
 template <int D>
 __global__ void __launch_bounds__(256) combine_kernel(DecodeArgs a) {
-  constexpr int PER = (D + 31) / 32;
+  grid_dep_wait();      // the partials of the decode kernel
+  grid_dep_launch();
+  constexpr int PER = D >= 32 ? D / 32 : 1;   // dimensions per lane
+  constexpr int LANES = D >= 32 ? 32 : D;     // lanes that hold dimensions
   const long long wid = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const long long U = (long long)a.B * a.Hkv;
@@ -570,44 +612,98 @@ __global__ void __launch_bounds__(256) combine_kernel(DecodeArgs a) {
   const int u = (int)(wid / a.R);
   const int r = (int)(wid % a.R);
   const int2 cr = a.unit_ctas[u];
-  if (cr.x >= cr.y) return;  // one CTA covered the unit and wrote out directly
-  // CTAs whose chunk range came out empty wrote no partial: skip them
   const long long total = *a.total_chunks;
-  auto nonempty = [&](int c) {
-    return total * c / a.grid < total * (c + 1) / a.grid;
+  if (cr.x >= cr.y) return;  // one CTA covered the unit and wrote out directly
+  const int n = cr.y - cr.x + 1;
+  // CTAs whose chunk range came out empty wrote no partial: weight 0
+  auto lse_of = [&](int j) -> float {
+    const int c = cr.x + j;
+    if (total * c / a.grid >= total * (c + 1) / a.grid) return -INFINITY;
+    return a.part_lse[((size_t)c + u) * a.R + r];
   };
   float M = -INFINITY;
-  for (int c = cr.x; c <= cr.y; ++c)
-    if (nonempty(c)) M = fmaxf(M, a.part_lse[((size_t)c + u) * a.R + r]);
+  for (int j = lane; j < n; j += 32) M = fmaxf(M, lse_of(j));
+#pragma unroll
+  for (int m = 16; m >= 1; m >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, m));
   const float Ms = (M == -INFINITY) ? 0.f : M;
+
+  const size_t stride = (size_t)a.R * D;  // between the partial rows of consecutive CTAs
+  const float* base = a.part_o + ((size_t)(cr.x + u) * a.R + r) * D + (size_t)lane * PER;
   float acc[PER];
 #pragma unroll
-  for (int k = 0; k < PER; ++k) acc[k] = 0.f;
+  for (int e = 0; e < PER; ++e) acc[e] = 0.f;
   float L = 0.f;
-  for (int c = cr.x; c <= cr.y; ++c) {
-    if (!nonempty(c)) continue;
-    const size_t sl = (size_t)c + u;
-    const float w = fast_exp2(a.part_lse[sl * a.R + r] - Ms);
+  for (int j0 = 0; j0 < n; j0 += 32) {
+    const float lj = (j0 + lane < n) ? lse_of(j0 + lane) : -INFINITY;
+    const float w = (lj == -INFINITY) ? 0.f : fast_exp2(lj - Ms);
     L += w;
-    const float* po = a.part_o + (sl * a.R + r) * D;
+    const int m = min(32, n - j0);
+    for (int k = 0; k < m; k += 4) {
+      float wk[4];
+      float x[4][PER];
 #pragma unroll
-    for (int k = 0; k < PER; ++k) {
-      const int d = lane + 32 * k;
-      if (d < D) acc[k] += w * po[d];
+      for (int i = 0; i < 4; ++i) {
+        const int kk = min(k + i, m - 1);             // past the end: reload a valid row, weight 0
+        wk[i] = __shfl_sync(0xffffffffu, w, kk);
+        if (k + i >= m) wk[i] = 0.f;
+        const float* src = base + (size_t)(j0 + kk) * stride;
+        if (lane < LANES) {
+          if constexpr (PER % 4 == 0) {
+#pragma unroll
+            for (int e = 0; e < PER; e += 4) {
+              const float4 v = *reinterpret_cast<const float4*>(src + e);
+              x[i][e] = v.x; x[i][e + 1] = v.y; x[i][e + 2] = v.z; x[i][e + 3] = v.w;
+            }
+          } else if constexpr (PER == 2) {
+            const float2 v = *reinterpret_cast<const float2*>(src);
+            x[i][0] = v.x; x[i][1] = v.y;
+          } else {
+            x[i][0] = src[0];
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < PER; ++e) x[i][e] = 0.f;
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int e = 0; e < PER; ++e) acc[e] += (wk[i] != 0.f) ? wk[i] * x[i][e] : 0.f;
     }
   }
+#pragma unroll
+  for (int m = 16; m >= 1; m >>= 1) L += __shfl_xor_sync(0xffffffffu, L, m);
+  if (lane >= LANES) return;
   const int b = u / a.Hkv, hk = u % a.Hkv;
   const int i = r / a.g;
   const int h = hk * a.g + r % a.g;
-  const size_t ob = (((size_t)b * a.T + i) * a.Hq + h) * D;
+  const size_t ob = (((size_t)b * a.T + i) * a.Hq + h) * D + (size_t)lane * PER;
   const float inv = (L > 0.f) ? 1.f / L : 0.f;
+  float o[PER];
 #pragma unroll
-  for (int k = 0; k < PER; ++k) {
-    const int d = lane + 32 * k;
-    if (d < D) {
-      const float o = acc[k] * inv;
-      if (a.out_bf16) reinterpret_cast<__nv_bfloat16*>(a.out)[ob + d] = __float2bfloat16_rn(o);
-      else reinterpret_cast<float*>(a.out)[ob + d] = o;
+  for (int e = 0; e < PER; ++e) o[e] = acc[e] * inv;
+  if (a.out_bf16) {
+    __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(a.out) + ob;
+    if constexpr (PER == 8) {
+      *reinterpret_cast<uint4*>(dst) = make_uint4(pack_bf16(o[0], o[1]), pack_bf16(o[2], o[3]),
+                                                  pack_bf16(o[4], o[5]), pack_bf16(o[6], o[7]));
+    } else if constexpr (PER == 4) {
+      *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16(o[0], o[1]), pack_bf16(o[2], o[3]));
+    } else if constexpr (PER == 2) {
+      *reinterpret_cast<uint32_t*>(dst) = pack_bf16(o[0], o[1]);
+    } else {
+      dst[0] = __float2bfloat16_rn(o[0]);
+    }
+  } else {
+    float* dst = reinterpret_cast<float*>(a.out) + ob;
+    if constexpr (PER % 4 == 0) {
+#pragma unroll
+      for (int e = 0; e < PER; e += 4)
+        *reinterpret_cast<float4*>(dst + e) = make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]);
+    } else if constexpr (PER == 2) {
+      *reinterpret_cast<float2*>(dst) = make_float2(o[0], o[1]);
+    } else {
+      dst[0] = o[0];
     }
   }
 }
@@ -641,13 +737,11 @@ cudaError_t launch_one(const DecodeArgs& a, int nrg, int cfg_idx, cudaStream_t s
     if (e != cudaSuccess) return e;
     flag.fetch_or(bit);
   }
-  kern<<<a.grid, (ncw + 1) * 32, smem, st>>>(a, nrg);
-  e = cudaGetLastError();
+  e = launch_pdl(kern, dim3(a.grid), dim3((ncw + 1) * 32), smem, st, a, nrg);
   if (e != cudaSuccess) return e;
   const long long warps = (long long)a.B * a.Hkv * a.R;
   const int cblocks = (int)((warps * 32 + 255) / 256);
-  combine_kernel<D><<<cblocks, 256, 0, st>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(combine_kernel<D>, dim3(cblocks), dim3(256), 0, st, a);
 }
 
 template <typename T, int D, bool PAGED>

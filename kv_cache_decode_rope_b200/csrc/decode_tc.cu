@@ -105,16 +105,17 @@ __device__ __forceinline__ void tc_loader(const DecodeArgs& a, const int* sPrefi
     if (ch >= kend) return -1;
     return a.block_table[(size_t)b * a.max_pages_per_seq + (ch * kChunk) / a.page_size];
   };
-  while (c.x < x1 && !failed) {
-    const int nb = sPrefix[c.b + 1] - sPrefix[c.b];
-    const int kend = (int)min((long long)nb, c.k0 + (x1 - c.x));
+  for (; c.x < x1 && !failed; next_unit(a, c, seg_of(a, sPrefix, c, x1))) {
+    const Seg sg = seg_of(a, sPrefix, c, x1);
+    if (sg.empty()) continue;
+    const int kend = sg.kend;
     // two 32-chunk windows of page ids, the second one loaded ahead of its use
-    int wbase = c.k0, win0 = -1, win1 = -1;
+    int wbase = sg.k0, win0 = -1, win1 = -1;
     if (PAGED) {
       win0 = page_of(c.b, wbase + lane, kend);
       win1 = page_of(c.b, wbase + 32 + lane, kend);
     }
-    for (int kk = c.k0; kk < kend; kk += CH, ++g) {
+    for (int kk = sg.k0; kk < kend; kk += CH, ++g) {
       if (PAGED && kk - wbase >= 32) {
         wbase += 32;
         win0 = win1;
@@ -151,9 +152,6 @@ __device__ __forceinline__ void tc_loader(const DecodeArgs& a, const int* sPrefi
       }
       __syncwarp();
     }
-    c.x += kend - c.k0;
-    c.k0 = 0;
-    if (++c.hk == a.Hkv) { c.hk = 0; ++c.b; }
   }
   if (lane == 0) {  // every issued copy lands before the CTA may exit
     for (int k = max(0, g - NSLOT); k < g; ++k)
@@ -232,6 +230,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *sTmem;
+  grid_dep_wait();      // q, the caches and the workspace are ready
+  grid_dep_launch();
 
   const long long total = (long long)a.Hkv * sPrefix[a.B];
   if (blockIdx.x == 0 && threadIdx.x == 0) *a.total_chunks = total;
@@ -254,10 +254,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         int g = 0, seg = 0;
         bool failed = false;
         SegState c = st;
-        while (c.x < x1 && !failed) {
-          const int nb = sPrefix[c.b + 1] - sPrefix[c.b];
-          const int kend = (int)min((long long)nb, c.k0 + (x1 - c.x));
-          const int n = (kend - c.k0 + CH - 1) / CH;
+        for (; c.x < x1 && !failed; next_unit(a, c, seg_of(a, sPrefix, c, x1))) {
+          const Seg sg = seg_of(a, sPrefix, c, x1);
+          if (sg.empty()) continue;
+          const int n = (sg.kend - sg.k0 + CH - 1) / CH;
           if (!mbar_wait(q_full, (uint32_t)seg & 1u, a.status)) { failed = true; break; }
           for (int k = 0; k < n; ++k) {
             const int gg = g + k;
@@ -281,9 +281,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           }
           g += n;
           ++seg;
-          c.x += kend - c.k0;
-          c.k0 = 0;
-          if (++c.hk == a.Hkv) { c.hk = 0; ++c.b; }
         }
         // every MMA this thread issued completes before the CTA frees TMEM
         tc_commit(&mma_done[0]);
@@ -299,10 +296,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         int g = 0;
         bool failed = false;
         SegState c = st;
-        while (c.x < x1 && !failed) {
-          const int nb = sPrefix[c.b + 1] - sPrefix[c.b];
-          const int kend = (int)min((long long)nb, c.k0 + (x1 - c.x));
-          const int n = (kend - c.k0 + CH - 1) / CH;
+        for (; c.x < x1 && !failed; next_unit(a, c, seg_of(a, sPrefix, c, x1))) {
+          const Seg sg = seg_of(a, sPrefix, c, x1);
+          if (sg.empty()) continue;
+          const int n = (sg.kend - sg.k0 + CH - 1) / CH;
           for (int k = 0; k < n && !failed; ++k) {
             const int gg = g + k;
             const int slot = gg % NV;
@@ -340,9 +337,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             if constexpr (C::STACK) tc_commit(&s_free[gg & 1]);   // P(gg) read: the S buffer is free
           }
           g += n;
-          c.x += kend - c.k0;
-          c.k0 = 0;
-          if (++c.hk == a.Hkv) { c.hk = 0; ++c.b; }
         }
         tc_commit(&mma_done[1]);
         mbar_wait(&mma_done[1], 0, a.status);
@@ -412,18 +406,19 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       int g = 0;
       bool failed = false;
       SegState c = st;
-      while (c.x < x1) {
-        const int nb = sPrefix[c.b + 1] - sPrefix[c.b];
+      for (; c.x < x1; next_unit(a, c, seg_of(a, sPrefix, c, x1))) {
+        const Seg sg = seg_of(a, sPrefix, c, x1);
+        if (sg.empty()) continue;
         const int Nb = Nb_cur;
         const int Lb = Nb - a.T;
-        const int kend = (int)min((long long)nb, c.k0 + (x1 - c.x));
-        const int n = (kend - c.k0 + CH - 1) / CH;
+        const int kend = sg.kend;
+        const int n = (kend - sg.k0 + CH - 1) / CH;
         const int u = c.b * a.Hkv + c.hk;
         const int vis = row_ok ? Lb + di + 1 : 0;            // visible tokens of this row
 
         // the next unit of this CTA's range, whose q is fetched during the last
         // stage of this one (the Q tile is free once that stage's QK is done)
-        const bool has_next = c.x + (kend - c.k0) < x1;
+        const bool has_next = next_has_work(a, sg, x1);
         const int nx_hk = (c.hk + 1 == a.Hkv) ? 0 : c.hk + 1;
         const int nx_b = (c.hk + 1 == a.Hkv) ? c.b + 1 : c.b;
         // length of the next unit's sequence, loaded now and used after this unit
@@ -432,8 +427,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         float m = -INFINITY, l = 0.f;
         for (int k = 0; k < n; ++k) {
           const int gg = g + k;
-          const int t0 = (c.k0 + k * CH) * kChunk;
-          const int nvalid = min(min(CH, kend - c.k0 - k * CH) * kChunk, Nb - t0);
+          const int t0 = (sg.k0 + k * CH) * kChunk;
+          const int nvalid = min(min(CH, kend - sg.k0 - k * CH) * kChunk, Nb - t0);
           const bool tail = (nvalid < ST) || (t0 + ST > Lb + 1);
           if (!failed && !mbar_wait(&s_full[gg & 1], (uint32_t)(gg >> 1) & 1u, a.status)) failed = true;
           tc_fence_after();
@@ -602,7 +597,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         const float L = w0 * h0.y + w1 * h1.y;
         const float inv = (L > 0.f) ? 1.f / L : 0.f;
         const float s0 = w0 * inv, s1 = w1 * inv;
-        const bool whole = (c.k0 == 0) && (kend == nb);
+        const bool whole = sg.whole();
         const long long slot_idx = (long long)blockIdx.x + u;
         const int h = c.hk * a.g + (row_ok ? qr % a.g : 0);
         float* orow = whole ? nullptr : a.part_o + ((size_t)slot_idx * a.R + qr) * TC_D;
@@ -661,16 +656,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         if (row_ok && !whole && hw == 0 && cs == 0)
           a.part_lse[(size_t)slot_idx * a.R + qr] = (L > 0.f) ? ms + fast_log2(L) : -INFINITY;
         if (threadIdx.x == 0) {
-          if (c.k0 == 0) a.unit_ctas[u].x = blockIdx.x;
-          if (kend == nb) a.unit_ctas[u].y = blockIdx.x;
+          if (sg.k0 == 0) a.unit_ctas[u].x = blockIdx.x;
+          if (sg.kend == sg.nb) a.unit_ctas[u].y = blockIdx.x;
         }
         tc_fence_before();  // the O reads above precede the next segment's first PV
         named_bar_sync(1, TC_SOFTMAX_THREADS);   // sML is reused by the next segment
 
         g += n;
-        c.x += kend - c.k0;
-        c.k0 = 0;
-        if (++c.hk == a.Hkv) { c.hk = 0; ++c.b; }
       }
     }
   }
@@ -731,12 +723,10 @@ cudaError_t launch_tc(const DecodeArgs& a, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     attr_done.fetch_or(bit);
   }
-  decode_tc_kernel<PAGED, M><<<a.grid, TC_THREADS, smem, st>>>(a, mk, mv);
-  e = cudaGetLastError();
+  e = launch_pdl(decode_tc_kernel<PAGED, M>, dim3(a.grid), dim3(TC_THREADS), smem, st, a, mk, mv);
   if (e != cudaSuccess) return e;
   const long long warps = (long long)a.B * a.Hkv * a.R;
-  combine_kernel<TC_D><<<(int)((warps * 32 + 255) / 256), 256, 0, st>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(combine_kernel<TC_D>, dim3((int)((warps * 32 + 255) / 256)), dim3(256), 0, st, a);
 }
 
 }  // namespace

@@ -99,6 +99,14 @@ __device__ __forceinline__ void bulk_g2s(void* smem_dst, const void* gmem_src, u
       : "memory");
 }
 
+// Programmatic dependent launch (see kvd_launch.h): wait until the previous
+// kernel on the stream has completed and its writes are visible; allow the
+// next kernel on the stream to begin its own set-up.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // 16-byte asynchronous copy global -> shared; `src_bytes` = 0 writes zeros
 // (the source is then not read).  Completion: cp_async_wait_all().
 __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src, uint32_t src_bytes) {
@@ -153,6 +161,12 @@ struct VecTraits<__nv_bfloat16> {
       f[k] = make_float2(__uint_as_float(w[k] << 16), __uint_as_float(w[k] & 0xffff0000u));
   }
 };
+
+// Two floats as one bf16x2 word (round to nearest even), `lo` in bits 0-15.
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return (uint32_t)__bfloat16_as_ushort(v.x) | ((uint32_t)__bfloat16_as_ushort(v.y) << 16);
+}
 
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
   return __ffma2_rn(a, b, c);

@@ -14,7 +14,7 @@ constexpr int kChunk = 16;        // tokens per work quantum (one page of 16, or
 constexpr int kMaxGrid = 1024;    // upper bound on decode CTAs; sizes the workspace
 constexpr int kMaxRows = 128;     // g * q_len rows per (sequence, kv head): tensor-core path
 constexpr int kMaxRowsCore = 64;  // ... on the CUDA-core path
-constexpr int kTcMinRows = 16;    // rows from which QK^T / PV run on the tensor cores
+constexpr int kTcMinRows = 8;     // rows from which QK^T / PV run on the tensor cores
 constexpr int kMaxBatch = 8192;   // sequences per call (per-CTA length scan lives in shared memory)
 
 struct AppendArgs {
@@ -42,7 +42,7 @@ struct DecodeArgs {
   float* part_o;      // [slots, R, D]
   float* part_lse;    // [slots, R]
   int2* unit_ctas;    // [U]: first and last CTA that touched each (sequence, kv head)
-  long long* total_chunks;  // written by CTA 0: chunks over all units (defines every CTA's range)
+  long long* total_chunks;  // written by CTA 0: length of the weighted chunk space (defines every CTA's range)
   int* status;
   int B, T, Hq, Hkv, g, R, D;
   int max_seq_len;                       // contiguous capacity
@@ -51,6 +51,7 @@ struct DecodeArgs {
   float qscale;                          // scale * log2(e)
   int out_bf16;
   int grid;                              // decode CTAs
+  int seg_cost;                          // virtual chunks charged per unit (set by the launch)
 };
 
 // Workspace carve-up, shared by kvd_workspace_size and the launch.
