@@ -21,9 +21,17 @@
  *   KVD_ERR_CUDA (details via cudaGetLastError in the caller's runtime).
  * - Problems only the device can see (a block-table entry outside
  *   [0, num_pages), a length beyond the cache capacity, a pipeline wait that
- *   ran out of its iteration limit) skip the affected access and OR a
+ *   ran out of its time limit) skip the affected access and OR a
  *   KVD_FLAG_* bit into *params->status when that pointer is non-NULL.  No
  *   kernel traps or asserts.
+ * - Stream order with programmatic dependent launch: every kernel of the
+ *   library may begin while the kernel before it on the stream finishes,
+ *   when that kernel allows early launch (the library's own kernels do).
+ *   Before waiting for it, a kernel reads only seq_lens and block_table;
+ *   q, k_new, v_new, the caches, out, the workspace and the status word are
+ *   touched only after that kernel has completed.  So a preceding kernel
+ *   that allows early launch must not write seq_lens or block_table; any
+ *   other preceding work is fully ordered as usual.
  *
  * Notation: B = batch, T = q_len (new tokens per sequence), Hq / Hkv = query /
  * key-value heads, g = Hq / Hkv, D = head_dim, L_b = seq_lens[b] = tokens
