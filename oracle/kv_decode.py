@@ -82,27 +82,43 @@ def round_store(x, dtype: str) -> np.ndarray:
 
 # ----------------------------------------------------------------------------
 # RoPE (ferric-core generate.rs, `rope_off_t` in `step_gpu`, `cpu::rope` in
-# `layer_cpu`): rotate each (j, j + D/2) pair by pos * theta_j.
+# `layer_cpu`): rotate each (j, j + D/2) pair by pos * theta_j.  The layout
+# variants (the ferrox-models index exports a `RopeLayout` type but defines no
+# member) are read as the two common ones: interleaved pairs (2j, 2j + 1), and a
+# rotary dimension r < D where only the first r elements rotate, with
+# theta_j = base^(-2j/r), and the other D - r pass through unchanged.
 # ----------------------------------------------------------------------------
 def rope_inv_freq(head_dim: int, base: float) -> np.ndarray:
-    """theta_j = base^(-2j/D) for j = 0 .. D/2-1."""
+    """theta_j = base^(-2j/D) for j = 0 .. D/2-1 (D = the rotated width)."""
     j = np.arange(head_dim // 2, dtype=F64)
     return np.power(F64(base), -2.0 * j / head_dim)
 
 
-def rope(x, positions, base: float) -> np.ndarray:
+def rope(x, positions, base: float, interleaved: bool = False, rotary_dim: int = 0) -> np.ndarray:
     """Rotate the last axis of ``x`` (length D) at the given absolute positions.
 
-    ``positions`` broadcasts against ``x.shape[:-1]``.
+    ``positions`` broadcasts against ``x.shape[:-1]``.  ``interleaved`` pairs
+    elements (2j, 2j + 1) instead of (j, j + r/2); ``rotary_dim`` = r (0 means
+    D) rotates the first r elements only.
     """
     x = np.asarray(x, dtype=F64)
     D = x.shape[-1]
-    half = D // 2
+    r = D if not rotary_dim else int(rotary_dim)
+    half = r // 2
     pos = np.asarray(positions, dtype=F64)
-    ang = pos[..., None] * rope_inv_freq(D, base)      # [..., D/2]
+    ang = pos[..., None] * rope_inv_freq(r, base)      # [..., r/2]
     c, s = np.cos(ang), np.sin(ang)
-    a, b = x[..., :half], x[..., half:]
-    return np.concatenate([a * c - b * s, a * s + b * c], axis=-1)
+    if interleaved:
+        a, b = x[..., 0:r:2], x[..., 1:r:2]
+    else:
+        a, b = x[..., :half], x[..., half:r]
+    ra, rb = a * c - b * s, a * s + b * c
+    out = x.copy()
+    if interleaved:
+        out[..., 0:r:2], out[..., 1:r:2] = ra, rb
+    else:
+        out[..., :half], out[..., half:r] = ra, rb
+    return out
 
 
 # ----------------------------------------------------------------------------
@@ -117,20 +133,22 @@ def _slot(b, p, cache_shape, block_table, page_size):
     return int(block_table[b, p // page_size]), p % page_size
 
 
-def rotate_new_tokens(q, k_new, v_new, seq_lens, base: float, dtype: str):
+def rotate_new_tokens(q, k_new, v_new, seq_lens, base: float, dtype: str,
+                      interleaved: bool = False, rotary_dim: int = 0):
     """q and k of the new tokens rotated at positions seq_lens[b] + i, and v,
     each rounded to the storage dtype: ``(q_rot, k_rot, v_stored)``."""
     q = np.asarray(q, F64)
     T = q.shape[1]
     pos = np.asarray(seq_lens, dtype=np.int64)[:, None] + np.arange(T)[None, :]  # [B, T]
-    q_rot = round_store(rope(q, pos[:, :, None], base), dtype)
-    k_rot = round_store(rope(np.asarray(k_new, F64), pos[:, :, None], base), dtype)
+    q_rot = round_store(rope(q, pos[:, :, None], base, interleaved, rotary_dim), dtype)
+    k_rot = round_store(rope(np.asarray(k_new, F64), pos[:, :, None], base, interleaved, rotary_dim),
+                        dtype)
     v_st = round_store(np.asarray(v_new, F64), dtype)
     return q_rot, k_rot, v_st
 
 
 def append_rope(q, k_new, v_new, k_cache, v_cache, seq_lens, base: float,
-                dtype: str, block_table=None):
+                dtype: str, block_table=None, interleaved: bool = False, rotary_dim: int = 0):
     """Rotate q and k_new at positions seq_lens[b] + i, store k and v.
 
     Returns ``(q_rot, k_cache, v_cache)`` as new fp64 arrays; q_rot and the
@@ -146,7 +164,8 @@ def append_rope(q, k_new, v_new, k_cache, v_cache, seq_lens, base: float,
     Hkv = k_new.shape[2]
     page_size = kc.shape[2] if block_table is not None else None
     pos = np.asarray(seq_lens, dtype=np.int64)[:, None] + np.arange(T)[None, :]  # [B, T]
-    q_rot, k_rot, v_st = rotate_new_tokens(q, k_new, v_new, seq_lens, base, dtype)
+    q_rot, k_rot, v_st = rotate_new_tokens(q, k_new, v_new, seq_lens, base, dtype,
+                                           interleaved, rotary_dim)
     for b in range(B):
         for i in range(T):
             p = int(pos[b, i])
@@ -233,7 +252,8 @@ def decode_attention(q_rot, k_cache, v_cache, seq_lens, scale: float,
 
 
 def full_causal_attention(q_raw, k_raw, v_raw, scale: float, base: float,
-                          dtype: str | None = None) -> np.ndarray:
+                          dtype: str | None = None, interleaved: bool = False,
+                          rotary_dim: int = 0) -> np.ndarray:
     """Non-cached recompute over whole sequences (generate.rs `forward_cpu`).
 
     ``q_raw [B, N, Hq, D]``, ``k_raw / v_raw [B, N, Hkv, D]`` hold the
@@ -249,8 +269,8 @@ def full_causal_attention(q_raw, k_raw, v_raw, scale: float, base: float,
     Hkv = k_raw.shape[2]
     g = Hq // Hkv
     pos = np.arange(N)[None, :, None]
-    q = rope(q_raw, pos, base)
-    k = rope(k_raw, pos, base)
+    q = rope(q_raw, pos, base, interleaved, rotary_dim)
+    k = rope(k_raw, pos, base, interleaved, rotary_dim)
     v = v_raw
     if dtype is not None:
         q, k, v = round_store(q, dtype), round_store(k, dtype), round_store(v, dtype)

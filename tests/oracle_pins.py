@@ -149,6 +149,79 @@ def pin_rope_complex_form(m):
                                np.concatenate([z.real, z.imag], -1), atol=1e-9)
 
 
+def pin_rope_interleaved_hand_case(m):
+    """Interleaved D=4, base 10000: pairs (0,1) and (2,3) with angles p*1 and p*0.01."""
+    got = m.rope(np.array([1.0, 0.0, 0.0, 0.0]), 1, 10000.0, interleaved=True)
+    np.testing.assert_allclose(got, [math.cos(1), math.sin(1), 0.0, 0.0], atol=1e-15)
+    got = m.rope(np.array([0.0, 0.0, 0.0, 2.0]), 100, 10000.0, interleaved=True)
+    np.testing.assert_allclose(got, [0.0, 0.0, -2 * math.sin(1), 2 * math.cos(1)], atol=1e-14)
+
+
+def pin_rope_interleaved_is_permuted_half_split(m):
+    """Interleaved pairing is half-split pairing of the vector whose first half
+    holds the even elements and second half the odd ones."""
+    r = rng(12)
+    for D in (2, 8, 64, 128):
+        x = r.standard_normal((5, D))
+        pos = r.integers(0, 131073, 5)
+        perm = np.concatenate([np.arange(0, D, 2), np.arange(1, D, 2)])
+        half = m.rope(x[:, perm], pos, 10000.0)
+        back = np.empty_like(half)
+        back[:, perm] = half
+        np.testing.assert_allclose(m.rope(x, pos, 10000.0, interleaved=True), back,
+                                   rtol=0, atol=1e-12)
+
+
+def pin_rope_partial_dims(m):
+    """rotary_dim r < D: the last D - r elements pass through untouched and the
+    first r are the full rotation of an r-vector (theta_j = base^(-2j/r)), for
+    both pairings; r = D is the plain rotation."""
+    r_ = rng(13)
+    for (D, r, inter) in [(8, 4, False), (8, 4, True), (64, 32, False), (128, 64, True),
+                          (128, 16, False)]:
+        x = r_.standard_normal((4, D))
+        pos = r_.integers(0, 131073, 4)
+        got = m.rope(x, pos, 10000.0, interleaved=inter, rotary_dim=r)
+        assert np.array_equal(got[:, r:], x[:, r:])
+        np.testing.assert_allclose(got[:, :r], m.rope(x[:, :r], pos, 10000.0, interleaved=inter),
+                                   rtol=0, atol=1e-12)
+        assert np.array_equal(m.rope(x, pos, 10000.0, inter, D), m.rope(x, pos, 10000.0, inter))
+    # closed form: D = 8, r = 4, base 100 -> theta = (1, 0.1), pair (0, 2) and (1, 3)
+    got = m.rope(np.array([0.0, 1.0, 0.0, 0.0, 5.0, 6.0, 7.0, 8.0]), 10, 100.0, rotary_dim=4)
+    np.testing.assert_allclose(got, [0.0, math.cos(1), 0.0, math.sin(1), 5.0, 6.0, 7.0, 8.0],
+                               atol=1e-14)
+
+
+def pin_rope_layouts_keep_relative_position(m):
+    """Every layout keeps <rope(q, p + s), rope(k, m + s)> a function of p - m."""
+    r = rng(14)
+    q, k = r.standard_normal(64), r.standard_normal(64)
+    for (inter, rd) in [(True, 0), (False, 32), (True, 16)]:
+        for (p, mm, s) in [(5, 3, 11), (131072, 7, 1000)]:
+            a = np.dot(m.rope(q, p + s, 10000.0, inter, rd), m.rope(k, mm + s, 10000.0, inter, rd))
+            b = np.dot(m.rope(q, p, 10000.0, inter, rd), m.rope(k, mm, 10000.0, inter, rd))
+            assert abs(a - b) <= 1e-9 * (1 + abs(b)), (inter, rd, p, mm, s)
+
+
+def pin_layouts_decode_equals_full_recompute(m):
+    """Cached decode with each RoPE layout equals the full recompute with it."""
+    for (inter, rd, D) in [(True, 0, 16), (False, 8, 16), (True, 16, 32)]:
+        B, N, Hq, Hkv = 2, 7, 4, 2
+        q, k, v = _raw_sequence(40 + D, B, N, Hq, Hkv, D)
+        sc = 1 / math.sqrt(D)
+        kc = np.full((B, Hkv, N + 1, D), np.nan)
+        vc = kc.copy()
+        outs = []
+        for L in range(N):
+            seq = np.full(B, L)
+            q_rot, kc, vc = m.append_rope(q[:, L:L + 1], k[:, L:L + 1], v[:, L:L + 1], kc, vc, seq,
+                                          10000.0, "f32", None, inter, rd)
+            outs.append(m.decode_attention(q_rot, kc, vc, seq, sc))
+        got = np.concatenate(outs, 1)
+        ref = m.full_causal_attention(q, k, v, sc, 10000.0, "f32", inter, rd)
+        assert np.max(np.abs(got - ref)) <= 1e-12
+
+
 # ------------------------------------------------------------------- attention
 def _attend_bruteforce(q_rows, K, V, scale, visible):
     """Pure-Python softmax attention, one element at a time."""

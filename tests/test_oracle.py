@@ -12,20 +12,41 @@ def test_oracle_pin(pin):
 
 
 # --- planted mistakes: each mutation of the oracle must fail at least one pin.
-def _rope_interleaved(x, positions, base):
+def _rope_interleaved(x, positions, base, interleaved=False, rotary_dim=0):
+    """Always pairs (2j, 2j + 1), whatever the layout asked for."""
+    return _orig_rope(x, positions, base, True, rotary_dim)
+
+
+def _rope_wrong_sign(x, positions, base, interleaved=False, rotary_dim=0):
+    return _orig_rope(x, -np.asarray(positions), base, interleaved, rotary_dim)
+
+
+def _rope_ignores_layout(x, positions, base, interleaved=False, rotary_dim=0):
+    return _orig_rope(x, positions, base)
+
+
+def _rope_partial_full_width_freq(x, positions, base, interleaved=False, rotary_dim=0):
+    """Partial rotation with theta_j = base^(-2j/D) instead of base^(-2j/r)."""
     x = np.asarray(x, np.float64)
     D = x.shape[-1]
-    ang = np.asarray(positions, np.float64)[..., None] * kv.rope_inv_freq(D, base)
-    c, s = np.cos(ang), np.sin(ang)
-    a, b = x[..., 0::2], x[..., 1::2]
-    out = np.empty_like(x)
-    out[..., 0::2] = a * c - b * s
-    out[..., 1::2] = a * s + b * c
+    r = rotary_dim or D
+    if r == D:
+        return _orig_rope(x, positions, base, interleaved)
+    scaled_base = float(base) ** (r / D)     # base'^(-2j/r) = base^(-2j/D)
+    out = x.copy()
+    out[..., :r] = _orig_rope(x[..., :r], positions, scaled_base, interleaved)
     return out
 
 
-def _rope_wrong_sign(x, positions, base):
-    return _orig_rope(x, -np.asarray(positions), base)
+def _rope_partial_rotates_all(x, positions, base, interleaved=False, rotary_dim=0):
+    """Rotates all D elements with the rotary-width frequencies of the first r."""
+    x = np.asarray(x, np.float64)
+    D = x.shape[-1]
+    r = rotary_dim or D
+    out = _orig_rope(x, positions, base, interleaved, r)
+    if r < D:
+        out[..., r:] = _orig_rope(x[..., r:], positions, base, interleaved)
+    return out
 
 
 def _inv_freq_off(head_dim, base):
@@ -67,6 +88,9 @@ _orig_gather = kv.gather_tokens
 MUTANTS = {
     "rope_interleaved_pairs": ("rope", _rope_interleaved),
     "rope_wrong_sign": ("rope", _rope_wrong_sign),
+    "rope_ignores_layout": ("rope", _rope_ignores_layout),
+    "rope_partial_full_width_freq": ("rope", _rope_partial_full_width_freq),
+    "rope_partial_rotates_all": ("rope", _rope_partial_rotates_all),
     "rope_freq_index_off": ("rope_inv_freq", _inv_freq_off),
     "attend_drops_scale": ("attend", _attend_no_scale),
     "attend_mask_off_by_one": ("attend", _attend_off_by_one),
