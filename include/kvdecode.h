@@ -103,6 +103,9 @@ typedef struct kvd_params {
   int max_pages_per_seq; /* paged: block_table row stride                             */
   int max_kv_len;        /* attention: host upper bound on L_b + T over the batch     */
   int* status;           /* optional device int, OR-ed with KVD_FLAG_* bits; may be 0 */
+  int rope_interleaved;  /* kv_append_rope: 0 = pairs (j, j + r/2), 1 = pairs (2j, 2j+1) */
+  int rotary_dim;        /* kv_append_rope: rotated width r (0 = head_dim); a multiple of
+                            16 <= head_dim; elements r .. D-1 are not rotated           */
 } kvd_params;
 
 /*
@@ -115,11 +118,16 @@ typedef struct kvd_params {
  * ferrum-sampler 0.7.0 README, "Key Optimizations" ("Batched RoPE: per-item
  * positions in single kernel launch").
  *
- * RoPE reading (the pages do not fix the pairing): half-split pairs (j, j+D/2)
- * for j < D/2 are rotated by angle (L_b+i) * rope_base^(-2j/D):
- *   (a, b) -> (a cos - b sin, a sin + b cos).
- * The angle and the rotation are evaluated in fp64 and rounded once to dtype
- * (round to nearest even).
+ * RoPE reading (the pages do not fix the pairing): with r = rotary_dim (0
+ * means D), the pairs (j, j + r/2) for j < r/2 are rotated by angle
+ * (L_b+i) * rope_base^(-2j/r):
+ *   (a, b) -> (a cos - b sin, a sin + b cos);
+ * rope_interleaved = 1 pairs (2j, 2j+1) instead (the ferrox-models index
+ * exports a `RopeLayout` type without defining its members; these are the two
+ * common layouts).  Elements r .. D-1 of q and k are not rotated.  The angle
+ * and the rotation are evaluated in fp64 and rounded once to dtype (round to
+ * nearest even).  KVD_ERR_UNSUPPORTED if rotary_dim is not 0 or a multiple of
+ * 16 in [16, D]; KVD_ERR_INVALID_ARG if rope_interleaved is not 0 or 1.
  *
  * q        in/out [B,T,Hq,D]: rotated in place.
  * k_new    in [B,T,Hkv,D]; v_new in [B,T,Hkv,D] (not modified).

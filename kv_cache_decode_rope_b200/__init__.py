@@ -45,7 +45,8 @@ def _stream(stream) -> int:
 
 def make_params(*, batch, num_heads, num_kv_heads, head_dim, q_len, dtype, scale=None,
                 rope_base=10000.0, out_dtype=None, max_seq_len=0, page_size=0, num_pages=0,
-                max_pages_per_seq=0, max_kv_len=0, status=None) -> Params:
+                max_pages_per_seq=0, max_kv_len=0, status=None, rope_interleaved=False,
+                rotary_dim=0) -> Params:
     """Build a ``kvd_params`` struct.  ``dtype``/``out_dtype`` are torch dtypes."""
     p = Params()
     p.batch, p.num_heads, p.num_kv_heads = batch, num_heads, num_kv_heads
@@ -57,6 +58,8 @@ def make_params(*, batch, num_heads, num_kv_heads, head_dim, q_len, dtype, scale
     p.max_seq_len, p.page_size, p.num_pages = max_seq_len, page_size, num_pages
     p.max_pages_per_seq, p.max_kv_len = max_pages_per_seq, max_kv_len
     p.status = None if status is None else _ptr(status)
+    p.rope_interleaved = 1 if rope_interleaved else 0
+    p.rotary_dim = int(rotary_dim)
     return p
 
 
@@ -80,9 +83,11 @@ def _geometry(q, k_cache, block_table):
 def append_rope(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor, k_cache: torch.Tensor,
                 v_cache: torch.Tensor, seq_lens: torch.Tensor, block_table: Optional[torch.Tensor] = None,
                 *, rope_base: float = 10000.0, status: Optional[torch.Tensor] = None,
-                stream=None) -> None:
+                stream=None, interleaved: bool = False, rotary_dim: int = 0) -> None:
     """``kv_append_rope``: rotate q in place, append rotated k and v at
-    positions seq_lens[b] + i.  Shapes as in include/kvdecode.h."""
+    positions seq_lens[b] + i.  Shapes as in include/kvdecode.h.
+    ``interleaved`` pairs elements (2j, 2j + 1); ``rotary_dim`` (0 = head_dim)
+    rotates the first rotary_dim elements only."""
     B, T, Hq, Hkv, D, paging = _geometry(q, k_cache, block_table)
     if k_new.shape != (B, T, Hkv, D) or v_new.shape != k_new.shape:
         raise ValueError("k_new / v_new must be [B, T, Hkv, D]")
@@ -92,7 +97,8 @@ def append_rope(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor, k_cac
     if seq_lens.dtype != torch.int32:
         raise TypeError("seq_lens must be int32")
     p = make_params(batch=B, num_heads=Hq, num_kv_heads=Hkv, head_dim=D, q_len=T, dtype=q.dtype,
-                    rope_base=rope_base, status=status, **paging)
+                    rope_base=rope_base, status=status, rope_interleaved=interleaved,
+                    rotary_dim=rotary_dim, **paging)
     rc = get_lib().kv_append_rope(ctypes.byref(p), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache),
                                   _ptr(v_cache), _ptr(seq_lens), _ptr(block_table), _stream(stream))
     _lib.check("kv_append_rope", rc)

@@ -47,6 +47,8 @@ class Params(ctypes.Structure):
         ("max_pages_per_seq", c_int),
         ("max_kv_len", c_int),
         ("status", c_void_p),
+        ("rope_interleaved", c_int),
+        ("rotary_dim", c_int),
     ]
 
 

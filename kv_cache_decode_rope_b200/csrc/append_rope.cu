@@ -6,13 +6,15 @@
 // ferrum-sampler 0.7.0 README ("Batched RoPE: per-item positions in single
 // kernel launch") every sequence of the batch carries its own position.
 //
-// One CTA per new token (b, i).  The CTA first evaluates the D/2 rotation
-// angles pos * base^(-2j/D) and their sine/cosine in fp64 into shared memory
+// One CTA per new token (b, i).  The CTA first evaluates the r/2 rotation
+// angles pos * base^(-2j/r) (r = rotated width, D unless a partial rotary
+// width is asked for) and their sine/cosine in fp64 into shared memory
 // (positions reach 1e5+, where an fp32 angle would be off by ~1e-2 rad).  Each
-// thread then rotates EPV half-split pairs (j, j + D/2) of one head row with
-// 16-byte loads and stores, in fp64, rounding once to the storage type, and
-// copies 16-byte pieces of v.  q is rotated in place; k and v go to the slot
-// of position seq_lens[b] + i.
+// thread then rotates the pairs held by 16-byte pieces of one head row, in
+// fp64, rounding once to the storage type: EPV half-split pairs (j, j + r/2)
+// from two pieces, or EPV/2 interleaved pairs (2j, 2j + 1) from one.  Pieces
+// past r are copied unrotated (k), or left in place (q), and v is copied.  q
+// is rotated in place; k and v go to the slot of position seq_lens[b] + i.
 #include <cuda_bf16.h>
 
 #include "kvd_device.cuh"
@@ -39,7 +41,6 @@ template <typename T, int D>
 __global__ void __launch_bounds__(256) append_rope_kernel(AppendArgs a) {
   constexpr int EPV = 16 / (int)sizeof(T);  // elements per 16-byte vector
   constexpr int HALF = D / 2;
-  constexpr int TPR = HALF / EPV;           // threads per rotated head row
   constexpr int VPR = D / EPV;              // 16-byte vectors per head row
   static_assert(HALF % EPV == 0, "half head must hold whole vectors");
 
@@ -51,8 +52,9 @@ __global__ void __launch_bounds__(256) append_rope_kernel(AppendArgs a) {
   const int i = blockIdx.x % a.T;
   const long long pos = (long long)a.seq_lens[b] + i;
 
-  for (int j = threadIdx.x; j < HALF; j += blockDim.x) {
-    const double inv_freq = pow(a.rope_base, -2.0 * (double)j / (double)D);
+  const int RH = a.rot / 2;                 // rotated pairs per head row
+  for (int j = threadIdx.x; j < RH; j += blockDim.x) {
+    const double inv_freq = pow(a.rope_base, -2.0 * (double)j / (double)a.rot);
     double s, c;
     sincos((double)pos * inv_freq, &s, &c);
     s_cos[j] = c;
@@ -88,41 +90,71 @@ __global__ void __launch_bounds__(256) append_rope_kernel(AppendArgs a) {
   __syncthreads();
 
   const long long tok = (long long)b * a.T + i;
-  const int n_rot = (a.Hq + a.Hkv) * TPR;
+  // per head row: RI rotation pieces, then (k only) PI pieces copied as they are
+  const int RI = a.interleaved ? a.rot / EPV : RH / EPV;
+  const int PI = (D - a.rot) / EPV;
+  const int n_q = a.Hq * RI;
+  const int n_rot = n_q + a.Hkv * (RI + PI);
   const int n_v = a.Hkv * VPR;
   for (int w = threadIdx.x; w < n_rot + n_v; w += blockDim.x) {
     if (w < n_rot) {
-      const int row = w / TPR;
-      const int j0 = (w % TPR) * EPV;
+      int it;
       const T* src;
       T* dst;
-      if (row < a.Hq) {
+      if (w < n_q) {
+        const int row = w / RI;
+        it = w % RI;
         T* qrow = reinterpret_cast<T*>(a.q) + (tok * a.Hq + row) * D;
         src = qrow;
         dst = qrow;
       } else {
-        const int hk = row - a.Hq;
+        const int w1 = w - n_q;
+        const int hk = w1 / (RI + PI);
+        it = w1 % (RI + PI);
         src = reinterpret_cast<const T*>(a.k_new) + (tok * a.Hkv + hk) * D;
         if (slot_base < 0) continue;
         dst = reinterpret_cast<T*>(a.k_cache) + slot_base + hk * head_stride;
       }
-      const uint4 ua = *reinterpret_cast<const uint4*>(src + j0);
-      const uint4 ub = *reinterpret_cast<const uint4*>(src + HALF + j0);
-      const T* xa = reinterpret_cast<const T*>(&ua);
-      const T* xb = reinterpret_cast<const T*>(&ub);
-      uint4 ra, rb;
-      T* ya = reinterpret_cast<T*>(&ra);
-      T* yb = reinterpret_cast<T*>(&rb);
-#pragma unroll
-      for (int e = 0; e < EPV; ++e) {
-        const double c = s_cos[j0 + e], s = s_sin[j0 + e];
-        const double va = Conv<T>::to_d(xa[e]), vb = Conv<T>::to_d(xb[e]);
-        // explicit roundings: a*c - b*s and a*s + b*c, each product rounded
-        ya[e] = Conv<T>::from_d(__dsub_rn(__dmul_rn(va, c), __dmul_rn(vb, s)));
-        yb[e] = Conv<T>::from_d(__dadd_rn(__dmul_rn(va, s), __dmul_rn(vb, c)));
+      if (it >= RI) {  // unrotated tail of k
+        const int e0 = a.rot + (it - RI) * EPV;
+        *reinterpret_cast<uint4*>(dst + e0) = *reinterpret_cast<const uint4*>(src + e0);
+        continue;
       }
-      *reinterpret_cast<uint4*>(dst + j0) = ra;
-      *reinterpret_cast<uint4*>(dst + HALF + j0) = rb;
+      // explicit roundings: a*c - b*s and a*s + b*c, each product rounded
+      if (!a.interleaved) {
+        const int j0 = it * EPV;
+        const uint4 ua = *reinterpret_cast<const uint4*>(src + j0);
+        const uint4 ub = *reinterpret_cast<const uint4*>(src + RH + j0);
+        const T* xa = reinterpret_cast<const T*>(&ua);
+        const T* xb = reinterpret_cast<const T*>(&ub);
+        uint4 ra, rb;
+        T* ya = reinterpret_cast<T*>(&ra);
+        T* yb = reinterpret_cast<T*>(&rb);
+#pragma unroll
+        for (int e = 0; e < EPV; ++e) {
+          const double c = s_cos[j0 + e], s = s_sin[j0 + e];
+          const double va = Conv<T>::to_d(xa[e]), vb = Conv<T>::to_d(xb[e]);
+          ya[e] = Conv<T>::from_d(__dsub_rn(__dmul_rn(va, c), __dmul_rn(vb, s)));
+          yb[e] = Conv<T>::from_d(__dadd_rn(__dmul_rn(va, s), __dmul_rn(vb, c)));
+        }
+        *reinterpret_cast<uint4*>(dst + j0) = ra;
+        *reinterpret_cast<uint4*>(dst + RH + j0) = rb;
+      } else {
+        const int e0 = it * EPV;  // elements e0 .. e0 + EPV - 1: pairs e0/2 ..
+        const uint4 u = *reinterpret_cast<const uint4*>(src + e0);
+        const T* x = reinterpret_cast<const T*>(&u);
+        uint4 ru;
+        T* y = reinterpret_cast<T*>(&ru);
+#pragma unroll
+        for (int e = 0; e < EPV; e += 2) {
+          const int j = e0 / 2 + e / 2;
+          const double c = s_cos[j], s = s_sin[j];
+          const double va = Conv<T>::to_d(x[e]), vb = Conv<T>::to_d(x[e + 1]);
+          y[e] = Conv<T>::from_d(__dsub_rn(__dmul_rn(va, c), __dmul_rn(vb, s)));
+          y[e + 1] = Conv<T>::from_d(__dadd_rn(__dmul_rn(va, s), __dmul_rn(vb, c)));
+        }
+        *reinterpret_cast<uint4*>(dst + e0) = ru;
+      }
     } else {
       if (slot_base < 0) continue;
       const int w2 = w - n_rot;

@@ -153,6 +153,9 @@ int kv_append_rope(const kvd_params* p, void* q, const void* k_new, const void* 
   rc = check_cache(p, paged);
   if (rc != KVD_OK) return rc;
   if (!std::isfinite(p->rope_base) || p->rope_base <= 0.f) return KVD_ERR_INVALID_ARG;
+  if (p->rope_interleaved != 0 && p->rope_interleaved != 1) return KVD_ERR_INVALID_ARG;
+  const int rot = p->rotary_dim == 0 ? p->head_dim : p->rotary_dim;
+  if (rot < 16 || rot > p->head_dim || rot % 16 != 0) return KVD_ERR_UNSUPPORTED;
   if (p->batch == 0 || p->q_len == 0) return KVD_OK;
   if ((long long)p->batch * p->q_len > INT32_MAX) return KVD_ERR_UNSUPPORTED;
   if (!q || !k_new || !v_new || !k_cache || !v_cache || !seq_lens) return KVD_ERR_INVALID_ARG;
@@ -178,6 +181,8 @@ int kv_append_rope(const kvd_params* p, void* q, const void* k_new, const void* 
   a.num_pages = p->num_pages;
   a.max_pages_per_seq = p->max_pages_per_seq;
   a.rope_base = (double)p->rope_base;
+  a.interleaved = p->rope_interleaved;
+  a.rot = rot;
   const cudaError_t e =
       launch_append(a, p->dtype == KVD_BF16, static_cast<cudaStream_t>(stream));
   if (e == cudaErrorNotSupported) return KVD_ERR_UNSUPPORTED;

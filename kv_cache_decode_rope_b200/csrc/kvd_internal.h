@@ -30,6 +30,8 @@ struct AppendArgs {
   int max_seq_len;
   int page_size, num_pages, max_pages_per_seq;
   double rope_base;
+  int interleaved;   // pairs (2j, 2j + 1) instead of (j, j + rot / 2)
+  int rot;           // rotated width (a multiple of 16, <= D)
 };
 
 struct DecodeArgs {

@@ -127,6 +127,10 @@ def test_paged_requires_table(lib):
 def test_append_validation(lib):
     def app(p, q=FAKE):
         return lib.kv_append_rope(ctypes.byref(p), q, FAKE, FAKE, FAKE, FAKE, FAKE, None, None)
+    assert app(params(rotary_dim=24)) == -2          # not a multiple of 16
+    assert app(params(rotary_dim=256)) == -2         # wider than head_dim
+    assert app(params(rotary_dim=8, head_dim=16)) == -2
+    assert app(params(rope_interleaved=2)) == -1
     assert app(params(rope_base=0.0)) == -1
     assert app(params(rope_base=float("inf"))) == -1
     assert app(params(head_dim=48)) == -2
