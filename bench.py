@@ -46,6 +46,9 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="CPU time budget of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--driver-layers", type=int, default=0,
+                    help="also time the decode-step driver (DecodeLoop) over this many layers of the "
+                         "workload's geometry: one token per step, graph replay vs eager calls")
     ap.add_argument("--launch", default="graph", choices=["graph", "eager"],
                     help="replay the step's library calls from CUDA graphs (default) or call them eagerly")
     return ap.parse_args()
@@ -67,12 +70,19 @@ def measured_peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
+# Sources that do not build the decode kernels (their changes leave a decode
+# launch's DRAM traffic as it was).
+NOT_DECODE = ("append_rope.cu", "kvd_static_ws.cu")
+
+
 def kernel_source_hash() -> str:
-    """Hash of the CUDA sources; a committed ncu figure is only valid for it."""
+    """Hash of the CUDA sources of the decode kernels and their launch; a
+    committed ncu traffic figure is only valid for it."""
     import glob
     import hashlib
     d = os.path.join(ROOT, "kv_cache_decode_rope_b200", "csrc")
     files = sorted(glob.glob(os.path.join(d, "*.cu*"))) + sorted(glob.glob(os.path.join(d, "*.h")))
+    files = [f for f in files if os.path.basename(f) not in NOT_DECODE]
     h = hashlib.sha256()
     for f in files:
         with open(f, "rb") as fh:
@@ -396,6 +406,47 @@ def workload_config(w, extra=None):
     return c
 
 
+def time_driver(w, n_layers: int, local: int, steps: int = 50) -> dict:
+    """Per-step device time of DecodeLoop over n_layers layers of the
+    workload's geometry: prefill of the workload's cache length through decode
+    steps, then single-token steps, replayed from the captured graph and
+    run as eager calls.  Caches are the driver's own (zero-filled, then written
+    by the prefill)."""
+    import torch
+    import kv_cache_decode_rope_b200 as kvd
+    dev = torch.device("cuda", local)
+    L0 = int(w.cache_len or w.len_range[1] // 4)
+    cap = L0 + 2 * (steps + 8)
+    res = {"layers": n_layers, "workload": w.name, "prefill_tokens": L0, "steps": steps}
+    gen = torch.Generator(device=dev).manual_seed(7)
+
+    def draw(T, H):
+        return torch.randn((n_layers, w.batch, T, H, w.head_dim), generator=gen, device=dev,
+                           dtype=torch.float32).to(w.torch_dtype)
+
+    for mode in ("graph", "eager"):
+        loop = kvd.DecodeLoop(n_layers=n_layers, batch=w.batch, num_heads=w.num_heads,
+                              num_kv_heads=w.num_kv_heads, head_dim=w.head_dim, capacity=cap,
+                              dtype=w.torch_dtype, paged=w.paged, page_size=w.page_size,
+                              rope_base=w.rope_base, graphs=(mode == "graph"), device=dev)
+        loop.prefill(draw(L0, w.num_heads), draw(L0, w.num_kv_heads), draw(L0, w.num_kv_heads))
+        ins = [(draw(1, w.num_heads), draw(1, w.num_kv_heads), draw(1, w.num_kv_heads))
+               for _ in range(steps + 4)]
+        for i in range(4):
+            loop.step(*ins[i])
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for i in range(4, steps + 4):
+            loop.step(*ins[i])
+        e1.record()
+        torch.cuda.synchronize(dev)
+        res[f"{mode}_us_per_step"] = round(e0.elapsed_time(e1) * 1e3 / steps, 2)
+        del loop
+    res["kernels_per_step"] = 3 * n_layers
+    return res
+
+
 def main():
     args = parse()
     rank, world, local = dist_env()
@@ -460,6 +511,8 @@ def main():
         "gpu_launches": 3 * K,
         "clocks": r["clocks"],
     }
+    if args.driver_layers > 0:
+        line["driver"] = time_driver(w, args.driver_layers, local)
     if rank == 0 and not args.no_cpu_baseline:
         v, cores, sample = oracle_sample(w, args.cpu_seconds, seed=1000 + w.config_id)
         line["cpu_baseline"] = {"value": round(v, 4), "unit": "GB/s", "cores": cores,

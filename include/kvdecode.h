@@ -193,6 +193,26 @@ KVD_API int decode_attention_paged(const kvd_params* p, const void* q, const voi
 KVD_API size_t kvd_workspace_size(const kvd_params* p);
 
 /*
+ * kvd_decode_step -- one layer's whole decode step: kv_append_rope, then
+ * decode_attention (block_table == NULL) or decode_attention_paged.
+ *
+ * The loop of ferric-core 0.1.0, examples/generate.rs, `step_gpu` (rope the
+ * new tokens, extend the caches, attend) in one call, so that a step of every
+ * layer can be captured into a CUDA graph call by call; the ferrum-sampler
+ * 0.7.0 README ("Performance") replays decode steps from CUDA graphs.
+ *
+ * Arguments as kv_append_rope followed by decode_attention[_paged] on the same
+ * q (rotated in place by the append), caches, seq_lens and block_table.  Both
+ * sets of checks run before anything is launched: any failed check returns
+ * its status and launches nothing.  seq_lens is not advanced: the caller adds
+ * q_len before the next step.
+ */
+KVD_API int kvd_decode_step(const kvd_params* p, void* q, const void* k_new, const void* v_new,
+                            void* k_cache, void* v_cache, const int32_t* seq_lens,
+                            const int32_t* block_table, void* out, void* workspace,
+                            size_t workspace_bytes, void* stream);
+
+/*
  * decode_attention_static -- decode_attention / decode_attention_paged for
  * callers that cannot allocate device memory.
  *

@@ -15,8 +15,8 @@ import torch
 from . import _lib
 from ._lib import KvdError, Params, get_lib  # noqa: F401
 
-__all__ = ["append_rope", "decode_attention", "decode_attention_paged", "workspace_size",
-           "make_params", "KvdError", "version"]
+__all__ = ["append_rope", "decode_attention", "decode_attention_paged", "decode_step",
+           "workspace_size", "make_params", "KvdError", "version", "DecodeLoop"]
 
 _DT = {torch.float32: _lib.KVD_F32, torch.bfloat16: _lib.KVD_BF16}
 
@@ -162,5 +162,44 @@ def decode_attention_paged(q, k_cache, v_cache, seq_lens, block_table, out=None,
                    stream=stream)
 
 
+def decode_step(q, k_new, v_new, k_cache, v_cache, seq_lens, block_table=None, out=None, *,
+                scale=None, max_kv_len=None, workspace=None, out_dtype=None, rope_base=10000.0,
+                interleaved=False, rotary_dim=0, status=None, stream=None) -> torch.Tensor:
+    """``kvd_decode_step``: append_rope then decode_attention[_paged] in one
+    library call (seq_lens is not advanced)."""
+    B, T, Hq, Hkv, D, paging = _geometry(q, k_cache, block_table)
+    if k_new.shape != (B, T, Hkv, D) or v_new.shape != k_new.shape:
+        raise ValueError("k_new / v_new must be [B, T, Hkv, D]")
+    for t in (k_new, v_new, k_cache, v_cache):
+        if t.dtype != q.dtype:
+            raise TypeError("q, k_new, v_new and the caches must share one dtype")
+    if seq_lens.dtype != torch.int32:
+        raise TypeError("seq_lens must be int32")
+    out_dtype = out.dtype if out is not None else (out_dtype or q.dtype)
+    if out is None:
+        out = torch.empty((B, T, Hq, D), dtype=out_dtype, device=q.device)
+    elif out.shape != (B, T, Hq, D):
+        raise ValueError("out must be [B, T, Hq, D]")
+    if max_kv_len is None:
+        max_kv_len = paging.get("max_seq_len") or paging["page_size"] * paging["max_pages_per_seq"]
+    p = make_params(batch=B, num_heads=Hq, num_kv_heads=Hkv, head_dim=D, q_len=T, dtype=q.dtype,
+                    scale=scale, out_dtype=out_dtype, max_kv_len=max_kv_len, status=status,
+                    rope_base=rope_base, rope_interleaved=interleaved, rotary_dim=rotary_dim,
+                    **paging)
+    lib = get_lib()
+    if workspace is None:
+        need = int(lib.kvd_workspace_size(ctypes.byref(p)))
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    nbytes = workspace.numel() * workspace.element_size()
+    rc = lib.kvd_decode_step(ctypes.byref(p), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache),
+                             _ptr(v_cache), _ptr(seq_lens), _ptr(block_table), _ptr(out),
+                             _ptr(workspace), nbytes, _stream(stream))
+    _lib.check("kvd_decode_step", rc)
+    return out
+
+
 def version() -> int:
     return int(get_lib().kvd_version())
+
+
+from .driver import DecodeLoop  # noqa: E402  (uses decode_step above)

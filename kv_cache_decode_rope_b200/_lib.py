@@ -64,6 +64,8 @@ SIGNATURES = {
     "decode_attention_static": (c_int, [PP, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                         c_void_p, c_void_p]),
     "kvd_workspace_size": (c_size_t, [PP]),
+    "kvd_decode_step": (c_int, [PP, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
     "kvd_status_string": (c_char_p, [c_int]),
     "kvd_version": (c_int, []),
 }

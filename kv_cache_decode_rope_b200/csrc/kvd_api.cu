@@ -60,9 +60,12 @@ int num_sms_current(int* dev_out) {
   return n;
 }
 
-int decode_common(const kvd_params* p, const void* q, const void* k_cache, const void* v_cache,
-                  const int32_t* seq_lens, const int32_t* block_table, void* out,
-                  void* workspace, size_t workspace_bytes, void* stream) {
+// Checks and argument set-up of a decode call; *nothing = true when there is
+// no work (empty batch or no new tokens).  No CUDA call except device queries.
+int prepare_decode(const kvd_params* p, const void* q, const void* k_cache, const void* v_cache,
+                   const int32_t* seq_lens, const int32_t* block_table, void* out,
+                   void* workspace, size_t workspace_bytes, DecodeArgs* args, bool* nothing) {
+  *nothing = false;
   int rc = check_common(p);
   if (rc != KVD_OK) return rc;
   const bool paged = block_table != nullptr;
@@ -70,7 +73,10 @@ int decode_common(const kvd_params* p, const void* q, const void* k_cache, const
   if (rc != KVD_OK) return rc;
   if (p->out_dtype != KVD_F32 && p->out_dtype != KVD_BF16) return KVD_ERR_INVALID_ARG;
   if (!std::isfinite(p->scale)) return KVD_ERR_INVALID_ARG;
-  if (p->batch == 0 || p->q_len == 0) return KVD_OK;  // nothing to attend
+  if (p->batch == 0 || p->q_len == 0) {  // nothing to attend
+    *nothing = true;
+    return KVD_OK;
+  }
   if (p->max_kv_len < 1) return KVD_ERR_INVALID_ARG;
   if (p->batch > kMaxBatch) return KVD_ERR_UNSUPPORTED;
   const int g = p->num_heads / p->num_kv_heads;
@@ -119,7 +125,77 @@ int decode_common(const kvd_params* p, const void* q, const void* k_cache, const
   a.out_bf16 = p->out_dtype == KVD_BF16;
   a.grid = decode_grid(p->batch, p->num_kv_heads, p->max_kv_len, sms, p->head_dim,
                              p->dtype == KVD_BF16, (int)R);
+  *args = a;
+  return KVD_OK;
+}
+
+int run_decode(const kvd_params* p, const DecodeArgs& a, void* stream) {
   const cudaError_t e = launch_decode(a, p->dtype == KVD_BF16, static_cast<cudaStream_t>(stream));
+  if (e == cudaErrorNotSupported) return KVD_ERR_UNSUPPORTED;
+  return e == cudaSuccess ? KVD_OK : KVD_ERR_CUDA;
+}
+
+int decode_common(const kvd_params* p, const void* q, const void* k_cache, const void* v_cache,
+                  const int32_t* seq_lens, const int32_t* block_table, void* out,
+                  void* workspace, size_t workspace_bytes, void* stream) {
+  DecodeArgs a{};
+  bool nothing = false;
+  const int rc = prepare_decode(p, q, k_cache, v_cache, seq_lens, block_table, out, workspace,
+                                workspace_bytes, &a, &nothing);
+  if (rc != KVD_OK || nothing) return rc;
+  return run_decode(p, a, stream);
+}
+
+// Checks and argument set-up of an append call (as prepare_decode).
+int prepare_append(const kvd_params* p, void* q, const void* k_new, const void* v_new,
+                   void* k_cache, void* v_cache, const int32_t* seq_lens,
+                   const int32_t* block_table, AppendArgs* args, bool* nothing) {
+  *nothing = false;
+  int rc = check_common(p);
+  if (rc != KVD_OK) return rc;
+  const bool paged = block_table != nullptr;
+  rc = check_cache(p, paged);
+  if (rc != KVD_OK) return rc;
+  if (!std::isfinite(p->rope_base) || p->rope_base <= 0.f) return KVD_ERR_INVALID_ARG;
+  if (p->rope_interleaved != 0 && p->rope_interleaved != 1) return KVD_ERR_INVALID_ARG;
+  const int rot = p->rotary_dim == 0 ? p->head_dim : p->rotary_dim;
+  if (rot < 16 || rot > p->head_dim || rot % 16 != 0) return KVD_ERR_UNSUPPORTED;
+  if (p->batch == 0 || p->q_len == 0) {
+    *nothing = true;
+    return KVD_OK;
+  }
+  if ((long long)p->batch * p->q_len > INT32_MAX) return KVD_ERR_UNSUPPORTED;
+  if (!q || !k_new || !v_new || !k_cache || !v_cache || !seq_lens) return KVD_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) ||
+      !aligned16(v_cache))
+    return KVD_ERR_INVALID_ARG;
+  AppendArgs a{};
+  a.q = q;
+  a.k_new = k_new;
+  a.v_new = v_new;
+  a.k_cache = k_cache;
+  a.v_cache = v_cache;
+  a.seq_lens = seq_lens;
+  a.block_table = block_table;
+  a.status = p->status;
+  a.B = p->batch;
+  a.T = p->q_len;
+  a.Hq = p->num_heads;
+  a.Hkv = p->num_kv_heads;
+  a.D = p->head_dim;
+  a.max_seq_len = p->max_seq_len;
+  a.page_size = p->page_size;
+  a.num_pages = p->num_pages;
+  a.max_pages_per_seq = p->max_pages_per_seq;
+  a.rope_base = (double)p->rope_base;
+  a.interleaved = p->rope_interleaved;
+  a.rot = rot;
+  *args = a;
+  return KVD_OK;
+}
+
+int run_append(const kvd_params* p, const AppendArgs& a, void* stream) {
+  const cudaError_t e = launch_append(a, p->dtype == KVD_BF16, static_cast<cudaStream_t>(stream));
   if (e == cudaErrorNotSupported) return KVD_ERR_UNSUPPORTED;
   return e == cudaSuccess ? KVD_OK : KVD_ERR_CUDA;
 }
@@ -147,46 +223,30 @@ extern "C" {
 int kv_append_rope(const kvd_params* p, void* q, const void* k_new, const void* v_new,
                    void* k_cache, void* v_cache, const int32_t* seq_lens,
                    const int32_t* block_table, void* stream) {
-  int rc = check_common(p);
-  if (rc != KVD_OK) return rc;
-  const bool paged = block_table != nullptr;
-  rc = check_cache(p, paged);
-  if (rc != KVD_OK) return rc;
-  if (!std::isfinite(p->rope_base) || p->rope_base <= 0.f) return KVD_ERR_INVALID_ARG;
-  if (p->rope_interleaved != 0 && p->rope_interleaved != 1) return KVD_ERR_INVALID_ARG;
-  const int rot = p->rotary_dim == 0 ? p->head_dim : p->rotary_dim;
-  if (rot < 16 || rot > p->head_dim || rot % 16 != 0) return KVD_ERR_UNSUPPORTED;
-  if (p->batch == 0 || p->q_len == 0) return KVD_OK;
-  if ((long long)p->batch * p->q_len > INT32_MAX) return KVD_ERR_UNSUPPORTED;
-  if (!q || !k_new || !v_new || !k_cache || !v_cache || !seq_lens) return KVD_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) ||
-      !aligned16(v_cache))
-    return KVD_ERR_INVALID_ARG;
   AppendArgs a{};
-  a.q = q;
-  a.k_new = k_new;
-  a.v_new = v_new;
-  a.k_cache = k_cache;
-  a.v_cache = v_cache;
-  a.seq_lens = seq_lens;
-  a.block_table = block_table;
-  a.status = p->status;
-  a.B = p->batch;
-  a.T = p->q_len;
-  a.Hq = p->num_heads;
-  a.Hkv = p->num_kv_heads;
-  a.D = p->head_dim;
-  a.max_seq_len = p->max_seq_len;
-  a.page_size = p->page_size;
-  a.num_pages = p->num_pages;
-  a.max_pages_per_seq = p->max_pages_per_seq;
-  a.rope_base = (double)p->rope_base;
-  a.interleaved = p->rope_interleaved;
-  a.rot = rot;
-  const cudaError_t e =
-      launch_append(a, p->dtype == KVD_BF16, static_cast<cudaStream_t>(stream));
-  if (e == cudaErrorNotSupported) return KVD_ERR_UNSUPPORTED;
-  return e == cudaSuccess ? KVD_OK : KVD_ERR_CUDA;
+  bool nothing = false;
+  const int rc = prepare_append(p, q, k_new, v_new, k_cache, v_cache, seq_lens, block_table, &a,
+                                &nothing);
+  if (rc != KVD_OK || nothing) return rc;
+  return run_append(p, a, stream);
+}
+
+int kvd_decode_step(const kvd_params* p, void* q, const void* k_new, const void* v_new,
+                    void* k_cache, void* v_cache, const int32_t* seq_lens,
+                    const int32_t* block_table, void* out, void* workspace,
+                    size_t workspace_bytes, void* stream) {
+  if (!p) return KVD_ERR_INVALID_ARG;
+  AppendArgs aa{};
+  DecodeArgs da{};
+  bool none_a = false, none_d = false;
+  int rc = prepare_append(p, q, k_new, v_new, k_cache, v_cache, seq_lens, block_table, &aa, &none_a);
+  if (rc != KVD_OK) return rc;
+  rc = prepare_decode(p, q, k_cache, v_cache, seq_lens, block_table, out, workspace,
+                      workspace_bytes, &da, &none_d);
+  if (rc != KVD_OK || none_a) return rc;
+  rc = run_append(p, aa, stream);
+  if (rc != KVD_OK || none_d) return rc;
+  return run_decode(p, da, stream);
 }
 
 int decode_attention(const kvd_params* p, const void* q, const void* k_cache,
