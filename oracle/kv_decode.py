@@ -41,6 +41,8 @@ q ``[B, T, Hq, D]``; k_new/v_new ``[B, T, Hkv, D]``; contiguous cache
 """
 from __future__ import annotations
 
+import math
+
 import numpy as np
 
 F64 = np.float64
@@ -249,6 +251,87 @@ def decode_attention(q_rot, k_cache, v_cache, seq_lens, scale: float,
         out[b] = decode_attention_rows(q_rot, k_cache, v_cache, seq_lens, scale, b,
                                        list(range(Hq)), block_table)
     return out
+
+
+# ----------------------------------------------------------------------------
+# Sequence-sharded decode: the split-K of "Flash Decoding" (ferrum-sampler 0.7.0
+# README, Key Optimizations) with the key ranges held by different devices.
+# Each shard returns, per query row, the attention over its own keys,
+# normalised, and the log-sum-exp of their scores; the merge weights shard s
+# by 2^(lse_s - max) and renormalises.  Log-sum-exps are in base 2, the unit
+# the kernels keep.
+# ----------------------------------------------------------------------------
+LN2 = math.log(2.0)
+
+
+def attend_partial(q_rows, K, V, scale: float, visible):
+    """Rows ``q_rows [R, D]`` against the first ``visible[r]`` keys of ``K, V
+    [N, D]``: ``(o [R, D], lse2 [R])`` with o the softmax-weighted mean of V
+    over those keys (0 when there are none) and lse2 = log2 sum_t exp(s_t),
+    s = scale q.k (-inf when there are none)."""
+    q_rows = np.asarray(q_rows, F64)
+    K = np.asarray(K, F64)
+    V = np.asarray(V, F64)
+    R, D = q_rows.shape
+    vis = np.asarray(visible)
+    o = np.zeros((R, D), F64)
+    lse = np.full(R, -np.inf)
+    if K.shape[0] == 0:
+        return o, lse
+    s = F64(scale) * (q_rows @ K.T)
+    t = np.arange(K.shape[0])[None, :]
+    s = np.where(t < vis[:, None], s, -np.inf)
+    for r in range(R):
+        if vis[r] <= 0:
+            continue
+        m = s[r].max()
+        p = np.exp(s[r] - m)
+        l = p.sum()
+        o[r] = (p @ V) / l
+        lse[r] = (m + math.log(l)) / LN2
+    return o, lse
+
+
+def decode_attention_shard(q_rot, k_local, v_local, seq_lens, shard_start, shard_lens,
+                           scale: float, block_table=None):
+    """One shard of a sequence-sharded decode step: ``(o [B, T, Hq, D],
+    lse2 [B, T, Hq])``.
+
+    The shard's cache holds, for sequence b, the tokens at global positions
+    shard_start[b] .. shard_start[b] + shard_lens[b] - 1 as its local tokens
+    0 .. shard_lens[b] - 1 (either layout).  New token i of sequence b (global
+    position seq_lens[b] + i) sees the local tokens whose global position is at
+    most seq_lens[b] + i.
+    """
+    q_rot = np.asarray(q_rot, F64)
+    B, T, Hq, D = q_rot.shape
+    Hkv = k_local.shape[1]
+    g = Hq // Hkv
+    o = np.zeros((B, T, Hq, D), F64)
+    lse = np.full((B, T, Hq), -np.inf)
+    for b in range(B):
+        n = int(shard_lens[b])
+        vis = np.clip(int(seq_lens[b]) + np.arange(T) + 1 - int(shard_start[b]), 0, n)
+        for hk in range(Hkv):
+            K = gather_tokens(k_local, b, hk, n, block_table)
+            V = gather_tokens(v_local, b, hk, n, block_table)
+            for h in range(hk * g, (hk + 1) * g):
+                o[b, :, h], lse[b, :, h] = attend_partial(q_rot[b, :, h], K, V, scale, vis)
+    return o, lse
+
+
+def merge_partials(o_parts, lse_parts) -> np.ndarray:
+    """``o_parts [S, ..., D]``, ``lse_parts [S, ...]`` (base 2) -> the merged
+    attention output ``[..., D]``: sum_s w_s o_s / sum_s w_s, w_s = 2^(lse_s - M),
+    M = max_s lse_s; shards with lse = -inf weigh 0."""
+    o_parts = np.asarray(o_parts, F64)
+    lse_parts = np.asarray(lse_parts, F64)
+    M = lse_parts.max(axis=0)
+    Ms = np.where(np.isfinite(M), M, 0.0)
+    w = np.where(np.isfinite(lse_parts), np.exp2(lse_parts - Ms), 0.0)
+    den = w.sum(axis=0)
+    num = (w[..., None] * o_parts).sum(axis=0)
+    return np.where(den[..., None] > 0, num / np.where(den > 0, den, 1.0)[..., None], 0.0)
 
 
 def full_causal_attention(q_raw, k_raw, v_raw, scale: float, base: float,

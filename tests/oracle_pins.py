@@ -417,4 +417,93 @@ def pin_causal_among_drafts(m):
     assert np.all(np.abs(a[0, 2] - b[0, 2]) > 1e-6)
 
 
+# ------------------------------------------------------------ sequence sharding
+def pin_attend_partial_closed_forms(m):
+    """One visible key: o = its v, lse2 = s / ln 2.  Two keys: lse2 = log2(e^s1 + e^s2).
+    None visible: o = 0, lse2 = -inf."""
+    q = np.array([[0.5, -1.0, 2.0, 0.25]])
+    K = np.array([[1.0, 2.0, 0.5, -1.0], [0.0, 1.0, 1.0, 3.0], [9.0, 9.0, 9.0, 9.0]])
+    V = np.array([[1.0, 2.0, 3.0, 4.0], [-1.0, 0.5, 0.0, 2.0], [7.0, 7.0, 7.0, 7.0]])
+    sc = 0.7
+    s1, s2 = sc * float(q[0] @ K[0]), sc * float(q[0] @ K[1])
+    o, lse = m.attend_partial(q, K, V, sc, [1])
+    np.testing.assert_allclose(o[0], V[0], atol=1e-15)
+    assert abs(lse[0] - s1 / math.log(2)) <= 1e-14
+    o, lse = m.attend_partial(q, K, V, sc, [2])
+    assert abs(lse[0] - math.log2(math.exp(s1) + math.exp(s2))) <= 1e-13
+    w1 = math.exp(s1) / (math.exp(s1) + math.exp(s2))
+    np.testing.assert_allclose(o[0], w1 * V[0] + (1 - w1) * V[1], atol=1e-14)
+    o, lse = m.attend_partial(q, K, V, sc, [0])
+    assert np.all(o == 0) and lse[0] == -np.inf
+
+
+def _split_cache(kc, vc, lens_total, cuts):
+    """Per-shard contiguous caches holding tokens [cuts[s], cuts[s+1]) of each sequence."""
+    B, Hkv, _, D = kc.shape
+    shards = []
+    for s in range(len(cuts) - 1):
+        start = np.array([min(cuts[s], n) for n in lens_total])
+        end = np.array([min(cuts[s + 1], n) for n in lens_total])
+        n_loc = end - start
+        cap = max(1, int(n_loc.max()))
+        k_loc = np.full((B, Hkv, cap, D), np.nan)
+        v_loc = np.full((B, Hkv, cap, D), np.nan)
+        for b in range(B):
+            k_loc[b, :, :n_loc[b]] = kc[b, :, start[b]:end[b]]
+            v_loc[b, :, :n_loc[b]] = vc[b, :, start[b]:end[b]]
+        shards.append((k_loc, v_loc, start, n_loc))
+    return shards
+
+
+def pin_shard_merge_equals_full_decode(m):
+    """Any cut of each sequence's keys into shards (empty shards and a shard of
+    new tokens only included), computed shard by shard and merged, equals the
+    unsharded decode; a single shard gives it directly with the brute-force
+    log-sum-exp."""
+    r = rng(15)
+    B, T, Hq, Hkv, D = 3, 3, 4, 2, 8
+    L = np.array([11, 4, 20])
+    N = L + T
+    q = r.standard_normal((B, T, Hq, D))
+    kc = r.standard_normal((B, Hkv, N.max() + 2, D))
+    vc = r.standard_normal((B, Hkv, N.max() + 2, D))
+    ref = m.decode_attention(q, kc, vc, L, 0.4)
+    for cuts in ([0, 30], [0, 5, 12, 30], [0, 0, 9, 9, 21, 22, 30], [0, 4, 5, 6, 7, 30]):
+        parts = [m.decode_attention_shard(q, k_loc, v_loc, L, start, n_loc, 0.4)
+                 for (k_loc, v_loc, start, n_loc) in _split_cache(kc, vc, N, cuts)]
+        got = m.merge_partials([p[0] for p in parts], [p[1] for p in parts])
+        assert np.max(np.abs(got - ref)) <= 1e-12, cuts
+    # one shard: lse equals the brute-force log2-sum-exp of the visible scores
+    o, lse = m.decode_attention_shard(q, kc, vc, L, np.zeros(B, int), N, 0.4)
+    b, i, h = 2, 1, 3
+    sc = [0.4 * float(q[b, i, h] @ kc[b, h // 2, t]) for t in range(L[b] + i + 1)]
+    assert abs(lse[b, i, h] - math.log2(sum(math.exp(x) for x in sc))) <= 1e-12
+    np.testing.assert_allclose(o, ref, atol=1e-12)
+
+
+def pin_shard_paged_equals_contiguous(m):
+    """A shard's paged cache (any page permutation) gives its contiguous result."""
+    r = rng(16)
+    B, T, Hq, Hkv, D, P = 2, 2, 4, 1, 8, 4
+    start = np.array([8, 3])
+    n_loc = np.array([9, 6])
+    L = np.array([15, 7])
+    q = r.standard_normal((B, T, Hq, D))
+    kc = r.standard_normal((B, Hkv, 12, D))
+    vc = r.standard_normal((B, Hkv, 12, D))
+    a = m.decode_attention_shard(q, kc, vc, L, start, n_loc, 0.3)
+    pages = 3
+    perm = r.permutation(B * pages)
+    bt = perm.reshape(B, pages)
+    kp = np.full((B * pages, Hkv, P, D), np.nan)
+    vp = kp.copy()
+    for b in range(B):
+        for t in range(12):
+            kp[bt[b, t // P], :, t % P] = kc[b, :, t]
+            vp[bt[b, t // P], :, t % P] = vc[b, :, t]
+    b_ = m.decode_attention_shard(q, kp, vp, L, start, n_loc, 0.3, bt)
+    np.testing.assert_allclose(a[0], b_[0], atol=1e-14)
+    np.testing.assert_allclose(a[1], b_[1], atol=1e-14)
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -81,7 +81,26 @@ def _gather_mod_heads(cache, b, h, n, block_table=None):
     return _orig_gather(cache, b, (h + 1) % cache.shape[1], n, block_table)
 
 
+def _merge_plain_mean(o_parts, lse_parts):
+    o = np.asarray(o_parts, np.float64)
+    live = np.isfinite(np.asarray(lse_parts))
+    return (o * live[..., None]).sum(0) / np.maximum(live.sum(0), 1)[..., None]
+
+
+def _attend_partial_natural_log(q_rows, K, V, scale, visible):
+    o, lse = _orig_attend_partial(q_rows, K, V, scale, visible)
+    return o, lse * kv.LN2
+
+
+def _shard_no_offset(q_rot, k_local, v_local, seq_lens, shard_start, shard_lens, scale,
+                     block_table=None):
+    return _orig_shard(q_rot, k_local, v_local, seq_lens, np.zeros_like(shard_start), shard_lens,
+                       scale, block_table)
+
+
 _orig_attend = kv.attend
+_orig_attend_partial = kv.attend_partial
+_orig_shard = kv.decode_attention_shard
 _orig_rope = kv.rope
 _orig_gather = kv.gather_tokens
 
@@ -97,6 +116,9 @@ MUTANTS = {
     "attend_k_v_swapped": ("attend", _attend_transposed),
     "bf16_truncates": ("bf16_round", _bf16_truncate),
     "wrong_kv_head": ("gather_tokens", _gather_mod_heads),
+    "merge_ignores_lse": ("merge_partials", _merge_plain_mean),
+    "partial_lse_natural_log": ("attend_partial", _attend_partial_natural_log),
+    "shard_mask_ignores_offset": ("decode_attention_shard", _shard_no_offset),
 }
 
 
