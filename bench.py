@@ -46,6 +46,10 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="CPU time budget of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--shard-seq", action="store_true",
+                    help="sequence-sharded decode: every rank holds 1/N of each sequence's "
+                         "positions; append + shard attention + all-gather of (o, lse) + merge "
+                         "(strong scaling; contiguous workloads)")
     ap.add_argument("--driver-layers", type=int, default=0,
                     help="also time the decode-step driver (DecodeLoop) over this many layers of the "
                          "workload's geometry: one token per step, graph replay vs eager calls")
@@ -458,6 +462,8 @@ def main():
         torch.cuda.set_device(local)
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local))
+    if args.shard_seq:
+        return main_sharded(args, rank, world, local)
     r = run_ours(args, rank, world, local)
     w = r["w"]
     K = args.steps
@@ -522,6 +528,122 @@ def main():
         torch.distributed.destroy_process_group()
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def main_sharded(args, rank, world, local):
+    """--shard-seq: the workload's sequences cut into `world` position ranges,
+    one per rank (kv_cache_decode_rope_b200.sharding); every step is the shard
+    append, the shard attention, the all-gather of (o, lse) and the merge."""
+    import torch
+    import kv_cache_decode_rope_b200 as kvd
+    from kv_cache_decode_rope_b200.sharding import gather_partials, shard_bounds
+    from kv_cache_decode_rope_b200.workloads import WORKLOADS, step_bytes
+    w = WORKLOADS[args.workload]
+    if w.paged or w.cache_len is None:
+        raise SystemExit("--shard-seq takes a contiguous workload with a fixed cache length")
+    dev = torch.device("cuda", local)
+    T, B, Hq, Hkv, D = w.q_len, w.batch, w.num_heads, w.num_kv_heads, w.head_dim
+    N = w.cache_len + T
+    C = ((N + world - 1) // world + 15) // 16 * 16          # positions per rank
+    gen = torch.Generator(device=dev).manual_seed(1000 + w.config_id + 7919 * rank)
+    rnd = lambda shape: torch.randn(shape, generator=gen, device=dev).to(w.torch_dtype)  # noqa: E731
+    k_loc, v_loc = rnd((B, Hkv, C, D)), rnd((B, Hkv, C, D))
+    q0, kn, vn = rnd((B, T, Hq, D)), rnd((B, T, Hkv, D)), rnd((B, T, Hkv, D))
+    seq = torch.full((B,), w.cache_len, dtype=torch.int32, device=dev)
+    start, lens = shard_bounds(seq, T, rank, C)
+    q = q0.clone()
+    o = torch.empty((B, T, Hq, D), dtype=torch.float32, device=dev)
+    lse = torch.empty((B, T, Hq), dtype=torch.float32, device=dev)
+    out = torch.empty((B, T, Hq, D), dtype=w.torch_dtype, device=dev)
+    ws = torch.empty(kvd.workspace_size(batch=B, num_heads=Hq, num_kv_heads=Hkv, head_dim=D,
+                                        q_len=T, dtype=w.torch_dtype), dtype=torch.uint8, device=dev)
+
+    def attend():
+        kvd.decode_attention_shard(q, k_loc, v_loc, seq, start, lens, scale=w.scale, max_kv_len=C,
+                                   workspace=ws, out=o, out_lse=lse)
+
+    def step():
+        q.copy_(q0)
+        kvd.append_rope_shard(q, kn, vn, k_loc, v_loc, seq, start, rope_base=w.rope_base)
+        attend()
+        if world > 1:
+            o_all, l_all = gather_partials(o, lse)
+            kvd.merge_partials(o_all, l_all, out=out)
+        else:
+            kvd.merge_partials(o[None], lse[None], out=out)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    run_step, run_attend = step, attend
+    graphs = []
+    if world == 1 and args.launch == "graph":     # collectives stay outside graphs
+        g1, g2 = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g1):
+            step()
+        with torch.cuda.graph(g2):
+            attend()
+        graphs = [g1, g2]
+        run_step, run_attend = g1.replay, g2.replay
+        for _ in range(3):
+            run_step()
+        torch.cuda.synchronize(dev)
+    K = args.steps
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(K):
+            run_step()
+        e1.record()
+        torch.cuda.synchronize(dev)
+    step_ms = e0.elapsed_time(e1) / K
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a0.record()
+    for _ in range(min(K, 200)):
+        run_attend()
+    a1.record()
+    torch.cuda.synchronize(dev)
+    att_ms = a0.elapsed_time(a1) / min(K, 200)
+    step_ms = reduce_max(step_ms, world)
+    att_ms = reduce_max(att_ms, world)
+    del graphs
+    esize = torch.empty((), dtype=w.torch_dtype).element_size()
+    seq_cpu = torch.full((B,), w.cache_len, dtype=torch.int64)
+    total = step_bytes(w, seq_cpu, esize)["step"]               # the whole job, all ranks
+    local_kv = int(lens.to(torch.int64).sum().item()) * Hkv * 2 * D * esize
+    peak, peak_kind = measured_peaks()
+    att_gbs = local_kv / (att_ms * 1e-3) / 1e9
+    line = {
+        "metric": METRIC,
+        "value": round(total / (step_ms * 1e-3) / 1e9, 1),
+        "unit": "GB/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": round(step_ms, 5), "us_per_step": round(step_ms * 1e3, 2),
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+        "dtype": "bf16" if w.dtype == "bf16" else "f32",
+        "data": "synthetic (seeded N(0,1) cache per rank, shapes of the workload)",
+        "config": workload_config(w, {
+            "parallelism": f"sequence-sharded x{world} ({C} positions per rank)",
+            "l2": "inputs larger than L2" if local_kv > 2 * L2_BYTES else "rank's shard fits L2",
+            "step": "kv_append_rope_shard + decode_attention_shard + all-gather + kvd_merge_partials",
+            "launch": "CUDA graph replay" if (world == 1 and args.launch == "graph")
+                      else "eager calls"}),
+        "roofline": {"bound": "hbm", "kernel": "decode_attention_shard (rank 0's shard)",
+                     "achieved": round(att_gbs, 1), "peak": peak,
+                     "peak_source": f"{peak_kind} hbm_gbs", "unit": "GB/s",
+                     "frac": round(att_gbs / peak, 4), "us_per_launch": round(att_ms * 1e3, 2),
+                     "algorithmic_bytes_per_launch": local_kv, "traffic": None},
+        "gpu_launches": 4 * K,      # append, shard attention, its split merge, shard merge
+        "clocks": clk.summary(),
+    }
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
 
 
 def main_reference(args, rank, world):

@@ -213,6 +213,70 @@ KVD_API int kvd_decode_step(const kvd_params* p, void* q, const void* k_new, con
                             size_t workspace_bytes, void* stream);
 
 /*
+ * Sequence-sharded decode (context parallelism): several devices each hold a
+ * range of every sequence's cached tokens, compute the attention of the new
+ * query tokens over their own range, exchange the per-row results and merge
+ * them.  This is the split-K of "Flash Decoding" (ferrum-sampler 0.7.0 README,
+ * "Key Optimizations") with the key ranges on different devices; ferrite's
+ * context-parallel decode is the same idea.
+ *
+ * A shard's cache holds, for sequence b, the tokens at global positions
+ * shard_start[b] .. shard_start[b] + shard_lens[b] - 1 as its local tokens
+ * 0 .. shard_lens[b] - 1, in either layout (max_seq_len / the block table
+ * describe the local cache).  seq_lens[b] stays the GLOBAL count of tokens
+ * before the step: new token i sits at global position seq_lens[b] + i.
+ */
+
+/*
+ * kv_append_rope_shard -- kv_append_rope for a shard: q and k of new token i
+ * are rotated at the global position seq_lens[b] + i; k and v are stored at the
+ * local slot seq_lens[b] + i - shard_start[b] when that slot lies inside the
+ * local cache; positions outside the shard's range are not stored (and not
+ * flagged: another shard holds them).  With k_cache == v_cache == NULL
+ * only q is rotated (k_new, v_new are then ignored): the shards that do not
+ * store the new tokens still need the rotated q.
+ */
+KVD_API int kv_append_rope_shard(const kvd_params* p, void* q, const void* k_new,
+                                 const void* v_new, void* k_cache, void* v_cache,
+                                 const int32_t* seq_lens, const int32_t* shard_start,
+                                 const int32_t* block_table, void* stream);
+
+/*
+ * decode_attention_shard -- one shard's part of a sequence-sharded decode.
+ *
+ * q        in [B,T,Hq,D], rotated.  New token i sees the local tokens whose
+ *          global position is at most seq_lens[b] + i (causal among drafts).
+ * shard_start, shard_lens in [B] int32 (device): the shard's token range of
+ *          each sequence; shard_lens[b] may be 0.
+ * block_table: NULL for the contiguous layout [B,Hkv,max_seq_len,D].
+ * out      out [B,T,Hq,D] fp32 (out_dtype must be KVD_F32): the attention
+ *          over this shard's visible tokens, normalised (0 if none).
+ * out_lse  out [B,T,Hq] fp32: log2 of the sum over those tokens of
+ *          exp(scale * q.k) (-inf if none).
+ * workspace: as decode_attention.  max_kv_len bounds shard_lens[b] (sizes the
+ *          grid).  Merging every shard's (out, out_lse) with
+ *          kvd_merge_partials gives decode_attention over the whole sequence.
+ */
+KVD_API int decode_attention_shard(const kvd_params* p, const void* q, const void* k_cache,
+                                   const void* v_cache, const int32_t* seq_lens,
+                                   const int32_t* shard_start, const int32_t* shard_lens,
+                                   const int32_t* block_table, float* out, float* out_lse,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * kvd_merge_partials -- merge S shards' results into the attention output.
+ *
+ * part_o   in [S,B,T,Hq,D] fp32, part_lse in [S,B,T,Hq] fp32 (base 2), stacked
+ *          in any shard order (device memory).
+ * out      out [B,T,Hq,D] in out_dtype:
+ *          sum_s w_s part_o[s] / sum_s w_s, w_s = 2^(part_lse[s] - max_s part_lse);
+ *          shards with lse = -inf weigh nothing (all -inf: 0).
+ * Uses batch, q_len, num_heads, head_dim and out_dtype of p.
+ */
+KVD_API int kvd_merge_partials(const kvd_params* p, const float* part_o, const float* part_lse,
+                               int num_shards, void* out, void* stream);
+
+/*
  * decode_attention_static -- decode_attention / decode_attention_paged for
  * callers that cannot allocate device memory.
  *

@@ -16,6 +16,7 @@ from . import _lib
 from ._lib import KvdError, Params, get_lib  # noqa: F401
 
 __all__ = ["append_rope", "decode_attention", "decode_attention_paged", "decode_step",
+           "append_rope_shard", "decode_attention_shard", "merge_partials",
            "workspace_size", "make_params", "KvdError", "version", "DecodeLoop"]
 
 _DT = {torch.float32: _lib.KVD_F32, torch.bfloat16: _lib.KVD_BF16}
@@ -195,6 +196,83 @@ def decode_step(q, k_new, v_new, k_cache, v_cache, seq_lens, block_table=None, o
                              _ptr(v_cache), _ptr(seq_lens), _ptr(block_table), _ptr(out),
                              _ptr(workspace), nbytes, _stream(stream))
     _lib.check("kvd_decode_step", rc)
+    return out
+
+
+def append_rope_shard(q, k_new, v_new, k_cache, v_cache, seq_lens, shard_start, block_table=None,
+                      *, rope_base: float = 10000.0, interleaved: bool = False, rotary_dim: int = 0,
+                      status=None, stream=None) -> None:
+    """``kv_append_rope_shard``: rotate q (and k) at the global positions
+    seq_lens[b] + i and store k, v at local slot seq_lens[b] + i - shard_start[b]
+    when the shard holds it.  ``k_cache = v_cache = None`` rotates q only."""
+    if shard_start.dtype != torch.int32 or seq_lens.dtype != torch.int32:
+        raise TypeError("seq_lens and shard_start must be int32")
+    rotate_only = k_cache is None and v_cache is None
+    B, T, Hq, D = q.shape
+    if rotate_only:
+        Hkv = k_new.shape[2] if k_new is not None else Hq
+        paging = dict(max_seq_len=1)
+        if block_table is not None:
+            raise ValueError("rotate-only mode takes no block_table")
+    else:
+        B, T, Hq, Hkv, D, paging = _geometry(q, k_cache, block_table)
+    p = make_params(batch=B, num_heads=Hq, num_kv_heads=Hkv, head_dim=D, q_len=T, dtype=q.dtype,
+                    rope_base=rope_base, status=status, rope_interleaved=interleaved,
+                    rotary_dim=rotary_dim, **paging)
+    rc = get_lib().kv_append_rope_shard(
+        ctypes.byref(p), _ptr(q), None if rotate_only else _ptr(k_new),
+        None if rotate_only else _ptr(v_new), None if rotate_only else _ptr(k_cache),
+        None if rotate_only else _ptr(v_cache), _ptr(seq_lens), _ptr(shard_start),
+        _ptr(block_table), _stream(stream))
+    _lib.check("kv_append_rope_shard", rc)
+
+
+def decode_attention_shard(q, k_cache, v_cache, seq_lens, shard_start, shard_lens, block_table=None,
+                           *, scale=None, max_kv_len=None, workspace=None, out=None, out_lse=None,
+                           status=None, stream=None):
+    """``decode_attention_shard``: this shard's (o [B,T,Hq,D] fp32, lse2 [B,T,Hq]
+    fp32) over its tokens of each sequence."""
+    B, T, Hq, Hkv, D, paging = _geometry(q, k_cache, block_table)
+    for t in (seq_lens, shard_start, shard_lens):
+        if t.dtype != torch.int32:
+            raise TypeError("seq_lens, shard_start and shard_lens must be int32")
+    if out is None:
+        out = torch.empty((B, T, Hq, D), dtype=torch.float32, device=q.device)
+    if out_lse is None:
+        out_lse = torch.empty((B, T, Hq), dtype=torch.float32, device=q.device)
+    if max_kv_len is None:
+        max_kv_len = paging.get("max_seq_len") or paging["page_size"] * paging["max_pages_per_seq"]
+    p = make_params(batch=B, num_heads=Hq, num_kv_heads=Hkv, head_dim=D, q_len=T, dtype=q.dtype,
+                    scale=scale, out_dtype=torch.float32, max_kv_len=max_kv_len, status=status,
+                    **paging)
+    lib = get_lib()
+    if workspace is None:
+        need = int(lib.kvd_workspace_size(ctypes.byref(p)))
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    nbytes = workspace.numel() * workspace.element_size()
+    rc = lib.decode_attention_shard(ctypes.byref(p), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                    _ptr(seq_lens), _ptr(shard_start), _ptr(shard_lens),
+                                    _ptr(block_table), _ptr(out), _ptr(out_lse), _ptr(workspace),
+                                    nbytes, _stream(stream))
+    _lib.check("decode_attention_shard", rc)
+    return out, out_lse
+
+
+def merge_partials(part_o, part_lse, out=None, *, out_dtype=None, stream=None) -> torch.Tensor:
+    """``kvd_merge_partials``: part_o [S,B,T,Hq,D] fp32, part_lse [S,B,T,Hq] fp32
+    -> the merged attention output [B,T,Hq,D]."""
+    S, B, T, Hq, D = part_o.shape
+    if part_lse.shape != (S, B, T, Hq) or part_o.dtype != torch.float32 \
+            or part_lse.dtype != torch.float32:
+        raise ValueError("part_o [S,B,T,Hq,D] and part_lse [S,B,T,Hq], both fp32")
+    out_dtype = out.dtype if out is not None else (out_dtype or torch.float32)
+    if out is None:
+        out = torch.empty((B, T, Hq, D), dtype=out_dtype, device=part_o.device)
+    p = make_params(batch=B, num_heads=Hq, num_kv_heads=Hq, head_dim=D, q_len=T,
+                    dtype=torch.float32, out_dtype=out_dtype)
+    rc = get_lib().kvd_merge_partials(ctypes.byref(p), _ptr(part_o), _ptr(part_lse), S, _ptr(out),
+                                      _stream(stream))
+    _lib.check("kvd_merge_partials", rc)
     return out
 
 

@@ -66,6 +66,12 @@ SIGNATURES = {
     "kvd_workspace_size": (c_size_t, [PP]),
     "kvd_decode_step": (c_int, [PP, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                 c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "kv_append_rope_shard": (c_int, [PP, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                     c_void_p, c_void_p, c_void_p, c_void_p]),
+    "decode_attention_shard": (c_int, [PP, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                       c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                       c_size_t, c_void_p]),
+    "kvd_merge_partials": (c_int, [PP, c_void_p, c_void_p, c_int, c_void_p, c_void_p]),
     "kvd_status_string": (c_char_p, [c_int]),
     "kvd_version": (c_int, []),
 }

@@ -64,29 +64,35 @@ __global__ void __launch_bounds__(256) append_rope_kernel(AppendArgs a) {
   // touching q, k/v, the caches or the status word
   grid_dep_wait();
 
-  // Where position `pos` of sequence b lives; -1 if it is outside the cache.
-  long long slot_base = -1;  // element offset of (kv head 0, pos); heads are `head_stride` apart
+  // Where position `pos` of sequence b lives (its local slot in a shard of a
+  // sequence-sharded cache); -1 if it is outside the cache.
+  const bool store = a.k_cache != nullptr;      // no caches: rotate q only
+  const long long lpos = a.shard_start ? pos - a.shard_start[b] : pos;
+  long long slot_base = -1;  // element offset of (kv head 0, lpos); heads are `head_stride` apart
   long long head_stride = 0;
-  if (pos >= 0) {
+  if (store && lpos >= 0) {
     if (a.block_table == nullptr) {
-      if (pos < a.max_seq_len) {
-        slot_base = ((long long)b * a.Hkv * a.max_seq_len + pos) * D;
+      if (lpos < a.max_seq_len) {
+        slot_base = ((long long)b * a.Hkv * a.max_seq_len + lpos) * D;
         head_stride = (long long)a.max_seq_len * D;
       }
     } else {
-      const long long lp = pos / a.page_size;
+      const long long lp = lpos / a.page_size;
       if (lp < a.max_pages_per_seq) {
         const int page = a.block_table[(long long)b * a.max_pages_per_seq + lp];
         if (page >= 0 && page < a.num_pages) {
-          slot_base = ((long long)page * a.Hkv * a.page_size + pos % a.page_size) * D;
+          slot_base = ((long long)page * a.Hkv * a.page_size + lpos % a.page_size) * D;
           head_stride = (long long)a.page_size * D;
         } else if (threadIdx.x == 0 && a.status) {
           atomicOr(a.status, KVD_FLAG_PAGE_OUT_OF_RANGE);
         }
       }
     }
+    // a shard stores only the positions inside its own range: elsewhere
+    // skipping is the normal case, not an error
+    if (slot_base < 0 && !a.shard_start && threadIdx.x == 0 && a.status)
+      atomicOr(a.status, KVD_FLAG_CAPACITY);
   }
-  if (slot_base < 0 && threadIdx.x == 0 && a.status) atomicOr(a.status, KVD_FLAG_CAPACITY);
   __syncthreads();
 
   const long long tok = (long long)b * a.T + i;
@@ -94,8 +100,8 @@ __global__ void __launch_bounds__(256) append_rope_kernel(AppendArgs a) {
   const int RI = a.interleaved ? a.rot / EPV : RH / EPV;
   const int PI = (D - a.rot) / EPV;
   const int n_q = a.Hq * RI;
-  const int n_rot = n_q + a.Hkv * (RI + PI);
-  const int n_v = a.Hkv * VPR;
+  const int n_rot = n_q + (store ? a.Hkv * (RI + PI) : 0);
+  const int n_v = store ? a.Hkv * VPR : 0;
   for (int w = threadIdx.x; w < n_rot + n_v; w += blockDim.x) {
     if (w < n_rot) {
       int it;

@@ -85,8 +85,17 @@ struct SegState {
   long long x;       // global chunk index of k0
 };
 
-// Per-sequence attended length N_b = L_b + T, clamped to the capacity.
+// Per-sequence attended length N_b = L_b + T, clamped to the capacity.  In
+// sequence-sharded mode: the tokens this shard holds, shard_lens[b].
 __device__ __forceinline__ int attended_len(const DecodeArgs& a, int b, bool flag) {
+  if (a.shard_lens) {
+    long long n = a.shard_lens[b];
+    if (n < 0 || n > a.cap_tokens) {
+      if (flag && a.status) atomicOr(a.status, KVD_FLAG_CAPACITY);
+      n = n < 0 ? 0 : (long long)a.cap_tokens;
+    }
+    return (int)n;
+  }
   long long L = a.seq_lens[b];
   long long N = L + a.T;
   if (L < 0 || N > a.cap_tokens) {
@@ -97,6 +106,17 @@ __device__ __forceinline__ int attended_len(const DecodeArgs& a, int b, bool fla
   return (int)N;
 }
 
+// Local position of the first new token of sequence b: token t (local) is
+// visible to new token i iff t < mask_base + i + 1.
+__device__ __forceinline__ int mask_base(const DecodeArgs& a, int b, int Nb) {
+  if (a.shard_start) return (int)max(-2147483647ll, (long long)a.seq_lens[b] - a.shard_start[b]);
+  return Nb - a.T;
+}
+
+// Chunks of a sequence's unit: at least one, so that a shard holding no token
+// of a sequence still writes its (empty) result.
+__device__ __forceinline__ int unit_chunks(int Nb) { return max(1, (Nb + kChunk - 1) / kChunk); }
+
 // The work split.  Each unit (sequence b, kv head) occupies seg_cost virtual
 // chunks followed by its ceil(N_b / 16) real chunks in one index space, units
 // in order (b, then kv head); CTA c takes the slice [total c / grid,
@@ -105,7 +125,7 @@ __device__ __forceinline__ int attended_len(const DecodeArgs& a, int b, bool fla
 // chunks.  Virtual chunks are never loaded.
 //
 // Block-wide exclusive scan of weighted chunks per sequence: sPrefix[b] = sum
-// over b' < b of (ceil(N_b' / 16) + seg_cost), sPrefix[B] = total.  All threads of the block
+// over b' < b of (max(1, ceil(N_b' / 16)) + seg_cost), sPrefix[B] = total.  All threads of the block
 // call it; `scratch` holds one int per warp.  Ends with __syncthreads.
 __device__ __forceinline__ void chunk_prefix_scan(const DecodeArgs& a, int* sPrefix, int* scratch) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -115,7 +135,7 @@ __device__ __forceinline__ void chunk_prefix_scan(const DecodeArgs& a, int* sPre
   const int hi = min(a.B, lo + per);
   int tsum = 0;
   for (int b = lo; b < hi; ++b)
-    tsum += (attended_len(a, b, blockIdx.x == 0) + kChunk - 1) / kChunk + a.seg_cost;
+    tsum += unit_chunks(attended_len(a, b, blockIdx.x == 0)) + a.seg_cost;
   int incl = tsum;
 #pragma unroll
   for (int m = 1; m < 32; m <<= 1) {
@@ -129,7 +149,7 @@ __device__ __forceinline__ void chunk_prefix_scan(const DecodeArgs& a, int* sPre
   int run = woff + incl - tsum;
   for (int b = lo; b < hi; ++b) {
     sPrefix[b] = run;
-    run += (attended_len(a, b, false) + kChunk - 1) / kChunk + a.seg_cost;
+    run += unit_chunks(attended_len(a, b, false)) + a.seg_cost;
   }
   if (hi == a.B && lo < hi) sPrefix[a.B] = run;
   __syncthreads();
@@ -282,13 +302,15 @@ __global__ void __launch_bounds__(NTW == 1 ? 288 : 160)
         T* dK = sK + (size_t)slot * G::STAGE_TOKENS * D;
         T* dV = sV + (size_t)slot * G::STAGE_TOKENS * D;
         if constexpr (!PAGED) {
-          const int ntok = min(nck * kChunk, Nb - t0);
-          const uint32_t bytes = (uint32_t)ntok * G::TOKEN_BYTES;
+          const int ntok = min(nck * kChunk, Nb - t0);   // <= 0: a shard without tokens here
+          const uint32_t bytes = ntok > 0 ? (uint32_t)ntok * G::TOKEN_BYTES : 0u;
           if (lane == 0) {
             mbar_arrive_expect_tx(&full[slot], 2 * bytes);
-            const size_t off = (((size_t)p.b * a.Hkv + p.hk) * a.max_seq_len + t0) * D;
-            bulk_g2s(dK, reinterpret_cast<const T*>(a.k_cache) + off, bytes, &full[slot]);
-            bulk_g2s(dV, reinterpret_cast<const T*>(a.v_cache) + off, bytes, &full[slot]);
+            if (bytes) {
+              const size_t off = (((size_t)p.b * a.Hkv + p.hk) * a.max_seq_len + t0) * D;
+              bulk_g2s(dK, reinterpret_cast<const T*>(a.k_cache) + off, bytes, &full[slot]);
+              bulk_g2s(dV, reinterpret_cast<const T*>(a.v_cache) + off, bytes, &full[slot]);
+            }
           }
         } else {
           // lane c < nck copies chunk c of the stage (16 tokens inside one page)
@@ -296,8 +318,8 @@ __global__ void __launch_bounds__(NTW == 1 ? 288 : 160)
           size_t off = 0;
           const int page =
               __shfl_sync(0xffffffffu, win0, kk - wbase + min(lane, G::STAGE_CHUNKS - 1));
-          if (lane < nck) {
-            const int tc = t0 + lane * kChunk;
+          const int tc = t0 + lane * kChunk;
+          if (lane < nck && tc < Nb) {
             const int ntok = min(kChunk, Nb - tc);
             if (page >= 0 && page < a.num_pages) {
               bytes = (uint32_t)ntok * G::TOKEN_BYTES;
@@ -351,7 +373,7 @@ __global__ void __launch_bounds__(NTW == 1 ? 288 : 160)
     const Seg sg = seg_of(a, sPrefix, c, x1);
     if (sg.empty()) continue;
     const int Nb = attended_len(a, c.b, false);
-    const int Lb = Nb - a.T;  // first new-token position (may be <= 0 after clamping)
+    const int Lb = mask_base(a, c.b, Nb);  // local position of the first new token (may be <= 0)
     const int kend = sg.kend;
     const int u = c.b * a.Hkv + c.hk;
 
@@ -578,9 +600,11 @@ __global__ void __launch_bounds__(NTW == 1 ? 288 : 160)
       if (whole) {
         const int i = rglob / a.g;
         const int h = c.hk * a.g + rglob % a.g;
-        const size_t oi = (((size_t)c.b * a.T + i) * a.Hq + h) * D + d;
+        const size_t row = ((size_t)c.b * a.T + i) * a.Hq + h;
+        const size_t oi = row * D + d;
         if (a.out_bf16) reinterpret_cast<__nv_bfloat16*>(a.out)[oi] = __float2bfloat16_rn(o);
         else reinterpret_cast<float*>(a.out)[oi] = o;
+        if (a.out_lse && d == 0) a.out_lse[row] = (L > 0.f) ? Ms + fast_log2(L) : -INFINITY;
       } else {
         a.part_o[((size_t)slot_idx * a.R + rglob) * D + d] = o;
         if (d == 0) a.part_lse[(size_t)slot_idx * a.R + rglob] = (L > 0.f) ? Ms + fast_log2(L) : -INFINITY;
@@ -677,8 +701,10 @@ __global__ void __launch_bounds__(256) combine_kernel(DecodeArgs a) {
   const int b = u / a.Hkv, hk = u % a.Hkv;
   const int i = r / a.g;
   const int h = hk * a.g + r % a.g;
-  const size_t ob = (((size_t)b * a.T + i) * a.Hq + h) * D + (size_t)lane * PER;
+  const size_t orow = ((size_t)b * a.T + i) * a.Hq + h;
+  const size_t ob = orow * D + (size_t)lane * PER;
   const float inv = (L > 0.f) ? 1.f / L : 0.f;
+  if (a.out_lse && lane == 0) a.out_lse[orow] = (L > 0.f) ? Ms + fast_log2(L) : -INFINITY;
   float o[PER];
 #pragma unroll
   for (int e = 0; e < PER; ++e) o[e] = acc[e] * inv;

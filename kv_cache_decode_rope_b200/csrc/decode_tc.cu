@@ -109,6 +109,7 @@ __device__ __forceinline__ void tc_loader(const DecodeArgs& a, const int* sPrefi
     const Seg sg = seg_of(a, sPrefix, c, x1);
     if (sg.empty()) continue;
     const int kend = sg.kend;
+    const int Nb = attended_len(a, c.b, false);   // chunks past it (a shard without tokens) are not loaded
     // two 32-chunk windows of page ids, the second one loaded ahead of its use
     int wbase = sg.k0, win0 = -1, win1 = -1;
     if (PAGED) {
@@ -130,7 +131,7 @@ __device__ __forceinline__ void tc_loader(const DecodeArgs& a, const int* sPrefi
       int page = -1;
       if (PAGED) page = __shfl_sync(0xffffffffu, win0, kk - wbase + min(lane, CH - 1));
       int row = -1;
-      if (lane < nck) {
+      if (lane < nck && (kk + lane) * kChunk < Nb) {
         const int tc = (kk + lane) * kChunk;
         if (!PAGED) {
           row = (int)(((long long)c.b * a.Hkv + c.hk) * a.max_seq_len + tc);
@@ -410,7 +411,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         const Seg sg = seg_of(a, sPrefix, c, x1);
         if (sg.empty()) continue;
         const int Nb = Nb_cur;
-        const int Lb = Nb - a.T;
+        const int Lb = mask_base(a, c.b, Nb);
         const int kend = sg.kend;
         const int n = (kend - sg.k0 + CH - 1) / CH;
         const int u = c.b * a.Hkv + c.hk;
@@ -653,8 +654,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             }
           }
         }
-        if (row_ok && !whole && hw == 0 && cs == 0)
-          a.part_lse[(size_t)slot_idx * a.R + qr] = (L > 0.f) ? ms + fast_log2(L) : -INFINITY;
+        if (row_ok && hw == 0 && cs == 0) {
+          const float lse = (L > 0.f) ? ms + fast_log2(L) : -INFINITY;
+          if (!whole) a.part_lse[(size_t)slot_idx * a.R + qr] = lse;
+          else if (a.out_lse) a.out_lse[ob / TC_D] = lse;
+        }
         if (threadIdx.x == 0) {
           if (sg.k0 == 0) a.unit_ctas[u].x = blockIdx.x;
           if (sg.kend == sg.nb) a.unit_ctas[u].y = blockIdx.x;

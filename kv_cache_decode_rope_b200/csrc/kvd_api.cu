@@ -149,7 +149,8 @@ int decode_common(const kvd_params* p, const void* q, const void* k_cache, const
 // Checks and argument set-up of an append call (as prepare_decode).
 int prepare_append(const kvd_params* p, void* q, const void* k_new, const void* v_new,
                    void* k_cache, void* v_cache, const int32_t* seq_lens,
-                   const int32_t* block_table, AppendArgs* args, bool* nothing) {
+                   const int32_t* block_table, AppendArgs* args, bool* nothing,
+                   bool rotate_only = false) {
   *nothing = false;
   int rc = check_common(p);
   if (rc != KVD_OK) return rc;
@@ -165,10 +166,15 @@ int prepare_append(const kvd_params* p, void* q, const void* k_new, const void* 
     return KVD_OK;
   }
   if ((long long)p->batch * p->q_len > INT32_MAX) return KVD_ERR_UNSUPPORTED;
-  if (!q || !k_new || !v_new || !k_cache || !v_cache || !seq_lens) return KVD_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) ||
-      !aligned16(v_cache))
-    return KVD_ERR_INVALID_ARG;
+  if (!q || !seq_lens || !aligned16(q)) return KVD_ERR_INVALID_ARG;
+  if (!rotate_only) {
+    if (!k_new || !v_new || !k_cache || !v_cache) return KVD_ERR_INVALID_ARG;
+    if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) || !aligned16(v_cache))
+      return KVD_ERR_INVALID_ARG;
+  } else {
+    k_new = v_new = nullptr;
+    k_cache = v_cache = nullptr;
+  }
   AppendArgs a{};
   a.q = q;
   a.k_new = k_new;
@@ -247,6 +253,64 @@ int kvd_decode_step(const kvd_params* p, void* q, const void* k_new, const void*
   rc = run_append(p, aa, stream);
   if (rc != KVD_OK || none_d) return rc;
   return run_decode(p, da, stream);
+}
+
+int kv_append_rope_shard(const kvd_params* p, void* q, const void* k_new, const void* v_new,
+                         void* k_cache, void* v_cache, const int32_t* seq_lens,
+                         const int32_t* shard_start, const int32_t* block_table, void* stream) {
+  if (!shard_start) return KVD_ERR_INVALID_ARG;
+  const bool rotate_only = k_cache == nullptr && v_cache == nullptr;
+  AppendArgs a{};
+  bool nothing = false;
+  const int rc = prepare_append(p, q, k_new, v_new, k_cache, v_cache, seq_lens, block_table, &a,
+                                &nothing, rotate_only);
+  if (rc != KVD_OK || nothing) return rc;
+  a.shard_start = shard_start;
+  return run_append(p, a, stream);
+}
+
+int decode_attention_shard(const kvd_params* p, const void* q, const void* k_cache,
+                           const void* v_cache, const int32_t* seq_lens,
+                           const int32_t* shard_start, const int32_t* shard_lens,
+                           const int32_t* block_table, float* out, float* out_lse,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+  if (!p || !shard_start || !shard_lens || !out_lse) return KVD_ERR_INVALID_ARG;
+  if (p->out_dtype != KVD_F32) return KVD_ERR_INVALID_ARG;   // partials are fp32
+  DecodeArgs a{};
+  bool nothing = false;
+  const int rc = prepare_decode(p, q, k_cache, v_cache, seq_lens, block_table, out, workspace,
+                                workspace_bytes, &a, &nothing);
+  if (rc != KVD_OK || nothing) return rc;
+  a.shard_start = shard_start;
+  a.shard_lens = shard_lens;
+  a.out_lse = out_lse;
+  return run_decode(p, a, stream);
+}
+
+int kvd_merge_partials(const kvd_params* p, const float* part_o, const float* part_lse,
+                       int num_shards, void* out, void* stream) {
+  int rc = check_common(p);
+  if (rc != KVD_OK) return rc;
+  if (p->out_dtype != KVD_F32 && p->out_dtype != KVD_BF16) return KVD_ERR_INVALID_ARG;
+  if (num_shards < 1) return KVD_ERR_INVALID_ARG;
+  const long long rows = (long long)p->batch * p->q_len * p->num_heads;
+  if (rows == 0) return KVD_OK;
+  if (!part_o || !part_lse || !out) return KVD_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(part_o) & 3u) || (reinterpret_cast<uintptr_t>(part_lse) & 3u) ||
+      !aligned16(out))
+    return KVD_ERR_INVALID_ARG;
+  if (rows * 32 > (long long)INT32_MAX * 8) return KVD_ERR_UNSUPPORTED;
+  MergeArgs a{};
+  a.part_o = part_o;
+  a.part_lse = part_lse;
+  a.out = out;
+  a.rows = rows;
+  a.shards = num_shards;
+  a.D = p->head_dim;
+  a.out_bf16 = p->out_dtype == KVD_BF16;
+  const cudaError_t e = launch_merge_shards(a, static_cast<cudaStream_t>(stream));
+  if (e == cudaErrorNotSupported) return KVD_ERR_UNSUPPORTED;
+  return e == cudaSuccess ? KVD_OK : KVD_ERR_CUDA;
 }
 
 int decode_attention(const kvd_params* p, const void* q, const void* k_cache,

@@ -32,6 +32,9 @@ struct AppendArgs {
   double rope_base;
   int interleaved;   // pairs (2j, 2j + 1) instead of (j, j + rot / 2)
   int rot;           // rotated width (a multiple of 16, <= D)
+  // Sequence-sharded mode: k and v of position p go to local slot
+  // p - shard_start[b] (null: slot p); null caches rotate q only.
+  const int32_t* shard_start;
 };
 
 struct DecodeArgs {
@@ -54,7 +57,23 @@ struct DecodeArgs {
   int out_bf16;
   int grid;                              // decode CTAs
   int seg_cost;                          // virtual chunks charged per unit (set by the launch)
+  // Sequence-sharded mode (all null otherwise): this cache holds the tokens at
+  // global positions shard_start[b] .. + shard_lens[b] - 1 of sequence b; the
+  // output is fp32 o in `out` plus the base-2 log-sum-exp of each row in out_lse.
+  const int32_t* shard_start;
+  const int32_t* shard_lens;
+  float* out_lse;
 };
+
+// Merge of sequence-sharded partials (kvd_merge_partials).
+struct MergeArgs {
+  const float* part_o;    // [shards, rows, D]
+  const float* part_lse;  // [shards, rows], base 2
+  void* out;              // [rows, D]
+  long long rows;         // B * T * Hq
+  int shards, D, out_bf16;
+};
+cudaError_t launch_merge_shards(const MergeArgs& a, cudaStream_t st);
 
 // Workspace carve-up, shared by kvd_workspace_size and the launch.
 struct WorkspaceLayout {
