@@ -150,12 +150,20 @@ def rotate_new_tokens(q, k_new, v_new, seq_lens, base: float, dtype: str,
 
 
 def append_rope(q, k_new, v_new, k_cache, v_cache, seq_lens, base: float,
-                dtype: str, block_table=None, interleaved: bool = False, rotary_dim: int = 0):
+                dtype: str, block_table=None, interleaved: bool = False, rotary_dim: int = 0,
+                cow_src=None):
     """Rotate q and k_new at positions seq_lens[b] + i, store k and v.
 
     Returns ``(q_rot, k_cache, v_cache)`` as new fp64 arrays; q_rot and the
     stored entries are rounded to ``dtype``.  Positions outside the cache are
     a caller error (IndexError).
+
+    Shared-prefix pages (the ferrox-models index's `prefix_cache`: sequences
+    that share a leading run of tokens share its pages): with ``cow_src``
+    (paged only), sequence b with cow_src[b] >= 0 first gets slots
+    0 .. seq_lens[b] % P - 1 of every kv head of page cow_src[b] copied, k and
+    v, into its own page block_table[b, seq_lens[b] // P] (copy on write of the
+    boundary page it shared); the source page is not modified.
     """
     q = np.asarray(q, F64)
     k_new = np.asarray(k_new, F64)
@@ -168,6 +176,15 @@ def append_rope(q, k_new, v_new, k_cache, v_cache, seq_lens, base: float,
     pos = np.asarray(seq_lens, dtype=np.int64)[:, None] + np.arange(T)[None, :]  # [B, T]
     q_rot, k_rot, v_st = rotate_new_tokens(q, k_new, v_new, seq_lens, base, dtype,
                                            interleaved, rotary_dim)
+    if cow_src is not None:
+        for b in range(B):
+            src = int(cow_src[b])
+            n = int(seq_lens[b]) % page_size
+            if src < 0 or n == 0:
+                continue
+            dst = int(block_table[b, int(seq_lens[b]) // page_size])
+            kc[dst, :, :n] = kc[src, :, :n]
+            vc[dst, :, :n] = vc[src, :, :n]
     for b in range(B):
         for i in range(T):
             p = int(pos[b, i])

@@ -417,6 +417,60 @@ def pin_causal_among_drafts(m):
     assert np.all(np.abs(a[0, 2] - b[0, 2]) > 1e-6)
 
 
+# ------------------------------------------------------------ shared prefixes
+def pin_copy_on_write_boundary_page(m):
+    """Two sequences share a prefix of 6 tokens (P = 4: one full page and a
+    boundary page half used).  Each gets a fresh boundary page by copy on
+    write; after the append, each decodes exactly as with private pages, and
+    the shared pages are unchanged."""
+    r = rng(17)
+    B, T, Hq, Hkv, D, P = 2, 2, 4, 2, 8, 4
+    shared = r.standard_normal((2, Hkv, P, D)), r.standard_normal((2, Hkv, P, D))  # pages 0, 1
+    kc = np.full((8, Hkv, P, D), np.nan)
+    vc = kc.copy()
+    kc[0:2], vc[0:2] = shared[0], shared[1]
+    L = np.array([6, 6])
+    bt = np.array([[0, 2, 3], [0, 4, 5]])          # boundary pages 2 and 4 are fresh
+    cow = np.array([1, 1])                          # both shared page 1
+    q, kn, vn = (r.standard_normal((B, T, Hq, D)), r.standard_normal((B, T, Hkv, D)),
+                 r.standard_normal((B, T, Hkv, D)))
+    q_rot, kc2, vc2 = m.append_rope(q, kn, vn, kc, vc, L, 10000.0, "f32", bt, cow_src=cow)
+    assert np.array_equal(kc2[0:2], kc[0:2]) and np.array_equal(vc2[0:2], vc[0:2])
+    # private reference: each sequence's own contiguous copy of the prefix
+    kp = np.full((B, Hkv, 12, D), np.nan)
+    vp = kp.copy()
+    for b in range(B):
+        for t in range(6):
+            kp[b, :, t] = kc[t // P, :, t % P]
+            vp[b, :, t] = vc[t // P, :, t % P]
+    q_p, kp2, vp2 = m.append_rope(q, kn, vn, kp, vp, L, 10000.0, "f32")
+    a = m.decode_attention(q_rot, kc2, vc2, L, 0.3, bt)
+    b_ = m.decode_attention(q_p, kp2, vp2, L, 0.3)
+    np.testing.assert_allclose(a, b_, atol=1e-14)
+    for b in range(B):   # the fresh page holds the copied slots, then the new tokens
+        np.testing.assert_array_equal(kc2[bt[b, 1], :, :2], kc[1, :, :2])
+    # no copy when the boundary falls on a page start
+    _, kc3, _ = m.append_rope(q, kn, vn, kc2, vc2, np.array([8, 8]), 10000.0, "f32", bt,
+                              cow_src=np.array([2, 4]))
+    assert np.array_equal(kc3[3, :, 2:], kc2[3, :, 2:], equal_nan=True)
+
+
+def pin_shared_prefix_decode(m):
+    """Sequences whose block tables share prefix pages decode as with private copies."""
+    r = rng(18)
+    B, T, Hq, Hkv, D, P = 3, 1, 4, 2, 8, 4
+    pool = 2 + 3 * 2
+    kc = r.standard_normal((pool, Hkv, P, D))
+    vc = r.standard_normal((pool, Hkv, P, D))
+    bt = np.array([[0, 1, 2, 3], [0, 1, 4, 5], [0, 1, 6, 7]])   # 8 shared tokens
+    L = np.array([10, 12, 8])
+    q = r.standard_normal((B, T, Hq, D))
+    kp = np.stack([np.concatenate([kc[bt[b, j]] for j in range(4)], axis=1) for b in range(B)])
+    vp = np.stack([np.concatenate([vc[bt[b, j]] for j in range(4)], axis=1) for b in range(B)])
+    np.testing.assert_allclose(m.decode_attention(q, kc, vc, L, 0.5, bt),
+                               m.decode_attention(q, kp, vp, L, 0.5), atol=1e-14)
+
+
 # ------------------------------------------------------------ sequence sharding
 def pin_attend_partial_closed_forms(m):
     """One visible key: o = its v, lse2 = s / ln 2.  Two keys: lse2 = log2(e^s1 + e^s2).

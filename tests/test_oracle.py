@@ -98,6 +98,12 @@ def _shard_no_offset(q_rot, k_local, v_local, seq_lens, shard_start, shard_lens,
                        scale, block_table)
 
 
+def _append_cow_skipped(*args, **kw):
+    kw.pop("cow_src", None)
+    return _orig_append(*args, **kw)
+
+
+_orig_append = kv.append_rope
 _orig_attend = kv.attend
 _orig_attend_partial = kv.attend_partial
 _orig_shard = kv.decode_attention_shard
@@ -119,6 +125,7 @@ MUTANTS = {
     "merge_ignores_lse": ("merge_partials", _merge_plain_mean),
     "partial_lse_natural_log": ("attend_partial", _attend_partial_natural_log),
     "shard_mask_ignores_offset": ("decode_attention_shard", _shard_no_offset),
+    "copy_on_write_skipped": ("append_rope", _append_cow_skipped),
 }
 
 
