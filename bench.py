@@ -405,6 +405,8 @@ def workload_config(w, extra=None):
          "head_dim": w.head_dim, "q_len": w.q_len,
          "cache": f"paged (page {w.page_size})" if w.paged else "contiguous",
          "cache_len": w.cache_len if w.cache_len is not None else f"log-uniform {w.len_range}"}
+    if w.shared_prefix:
+        c["shared_prefix"] = f"{w.shared_prefix} tokens in pages shared by every sequence"
     if extra:
         c.update(extra)
     return c

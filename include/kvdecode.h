@@ -213,6 +213,28 @@ KVD_API int kvd_decode_step(const kvd_params* p, void* q, const void* k_new, con
                             size_t workspace_bytes, void* stream);
 
 /*
+ * kv_append_rope_cow -- kv_append_rope on a paged cache whose sequences may
+ * share prefix pages, with copy on write of the shared boundary page.
+ *
+ * Sequences that start with the same tokens can point their block-table rows
+ * at the same physical pages (the ferrox-models index's `prefix_cache`: reuse
+ * the KV state of a shared leading subsequence instead of recomputing it);
+ * decode_attention_paged reads such pages like any other.  A page that is
+ * shared and only partly filled cannot take a sequence's new tokens: the
+ * caller (who owns page allocation) gives the sequence a fresh page in
+ * block_table[b][L_b / page_size] and passes the shared page's id in
+ * cow_src[b].  Before the new tokens land, slots 0 .. L_b % page_size - 1 of
+ * every kv head of page cow_src[b] are copied, k and v, into the fresh page;
+ * the shared page is not modified.  cow_src[b] < 0, or L_b a multiple of
+ * page_size, means no copy.  Otherwise as kv_append_rope (paged only); page ids
+ * outside [0, num_pages) skip the copy and flag KVD_FLAG_PAGE_OUT_OF_RANGE.
+ * cow_src in [B] int32, device memory; block_table required.
+ */
+KVD_API int kv_append_rope_cow(const kvd_params* p, void* q, const void* k_new, const void* v_new,
+                               void* k_cache, void* v_cache, const int32_t* seq_lens,
+                               const int32_t* block_table, const int32_t* cow_src, void* stream);
+
+/*
  * Sequence-sharded decode (context parallelism): several devices each hold a
  * range of every sequence's cached tokens, compute the attention of the new
  * query tokens over their own range, exchange the per-row results and merge

@@ -16,7 +16,7 @@ from . import _lib
 from ._lib import KvdError, Params, get_lib  # noqa: F401
 
 __all__ = ["append_rope", "decode_attention", "decode_attention_paged", "decode_step",
-           "append_rope_shard", "decode_attention_shard", "merge_partials",
+           "append_rope_cow", "append_rope_shard", "decode_attention_shard", "merge_partials",
            "workspace_size", "make_params", "KvdError", "version", "DecodeLoop"]
 
 _DT = {torch.float32: _lib.KVD_F32, torch.bfloat16: _lib.KVD_BF16}
@@ -197,6 +197,24 @@ def decode_step(q, k_new, v_new, k_cache, v_cache, seq_lens, block_table=None, o
                              _ptr(workspace), nbytes, _stream(stream))
     _lib.check("kvd_decode_step", rc)
     return out
+
+
+def append_rope_cow(q, k_new, v_new, k_cache, v_cache, seq_lens, block_table, cow_src, *,
+                    rope_base: float = 10000.0, interleaved: bool = False, rotary_dim: int = 0,
+                    status=None, stream=None) -> None:
+    """``kv_append_rope_cow``: append_rope on a paged cache, first copying the
+    slots before seq_lens[b] of shared page cow_src[b] (>= 0) into the
+    sequence's own page block_table[b, seq_lens[b] // page_size]."""
+    if cow_src.dtype != torch.int32:
+        raise TypeError("cow_src must be int32")
+    B, T, Hq, Hkv, D, paging = _geometry(q, k_cache, block_table)
+    p = make_params(batch=B, num_heads=Hq, num_kv_heads=Hkv, head_dim=D, q_len=T, dtype=q.dtype,
+                    rope_base=rope_base, status=status, rope_interleaved=interleaved,
+                    rotary_dim=rotary_dim, **paging)
+    rc = get_lib().kv_append_rope_cow(ctypes.byref(p), _ptr(q), _ptr(k_new), _ptr(v_new),
+                                      _ptr(k_cache), _ptr(v_cache), _ptr(seq_lens),
+                                      _ptr(block_table), _ptr(cow_src), _stream(stream))
+    _lib.check("kv_append_rope_cow", rc)
 
 
 def append_rope_shard(q, k_new, v_new, k_cache, v_cache, seq_lens, shard_start, block_table=None,

@@ -66,6 +66,8 @@ SIGNATURES = {
     "kvd_workspace_size": (c_size_t, [PP]),
     "kvd_decode_step": (c_int, [PP, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                 c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "kv_append_rope_cow": (c_int, [PP, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                   c_void_p, c_void_p, c_void_p, c_void_p]),
     "kv_append_rope_shard": (c_int, [PP, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                      c_void_p, c_void_p, c_void_p, c_void_p]),
     "decode_attention_shard": (c_int, [PP, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,

@@ -95,6 +95,32 @@ __global__ void __launch_bounds__(256) append_rope_kernel(AppendArgs a) {
   }
   __syncthreads();
 
+  // copy on write of a shared boundary page: the first token's CTA copies the
+  // slots before L_b into the sequence's own page (the new tokens go to later
+  // slots of that page, so the two never touch the same bytes)
+  if (a.cow_src && i == 0 && store) {
+    const int src = a.cow_src[b];
+    const long long L = pos;
+    const int n = (int)(L % a.page_size);
+    if (src >= 0 && n > 0) {
+      const long long lp = L / a.page_size;
+      const int dst = lp < a.max_pages_per_seq ? a.block_table[(long long)b * a.max_pages_per_seq + lp] : -1;
+      if (src < a.num_pages && dst >= 0 && dst < a.num_pages) {
+        const int per_tensor = a.Hkv * n * VPR;   // 16-byte pieces of one tensor
+        for (int e = threadIdx.x; e < 2 * per_tensor; e += blockDim.x) {
+          const int which = e / per_tensor, r = e % per_tensor;
+          const int hk = r / (n * VPR), slot = (r / VPR) % n, part = (r % VPR) * EPV;
+          T* cache = reinterpret_cast<T*>(which ? a.v_cache : a.k_cache);
+          const long long so = (((long long)src * a.Hkv + hk) * a.page_size + slot) * D + part;
+          const long long doff = (((long long)dst * a.Hkv + hk) * a.page_size + slot) * D + part;
+          *reinterpret_cast<uint4*>(cache + doff) = *reinterpret_cast<const uint4*>(cache + so);
+        }
+      } else if (threadIdx.x == 0 && a.status) {
+        atomicOr(a.status, KVD_FLAG_PAGE_OUT_OF_RANGE);
+      }
+    }
+  }
+
   const long long tok = (long long)b * a.T + i;
   // per head row: RI rotation pieces, then (k only) PI pieces copied as they are
   const int RI = a.interleaved ? a.rot / EPV : RH / EPV;

@@ -109,7 +109,9 @@ __device__ __forceinline__ void tc_loader(const DecodeArgs& a, const int* sPrefi
     const Seg sg = seg_of(a, sPrefix, c, x1);
     if (sg.empty()) continue;
     const int kend = sg.kend;
-    const int Nb = attended_len(a, c.b, false);   // chunks past it (a shard without tokens) are not loaded
+    // a shard holding no token of the sequence still has one (empty) chunk:
+    // it is not loaded; outside sharded mode every chunk holds tokens
+    const int Nb = a.shard_lens ? attended_len(a, c.b, false) : INT_MAX;
     // two 32-chunk windows of page ids, the second one loaded ahead of its use
     int wbase = sg.k0, win0 = -1, win1 = -1;
     if (PAGED) {

@@ -255,6 +255,19 @@ int kvd_decode_step(const kvd_params* p, void* q, const void* k_new, const void*
   return run_decode(p, da, stream);
 }
 
+int kv_append_rope_cow(const kvd_params* p, void* q, const void* k_new, const void* v_new,
+                       void* k_cache, void* v_cache, const int32_t* seq_lens,
+                       const int32_t* block_table, const int32_t* cow_src, void* stream) {
+  if (!block_table || !cow_src) return KVD_ERR_INVALID_ARG;
+  AppendArgs a{};
+  bool nothing = false;
+  const int rc = prepare_append(p, q, k_new, v_new, k_cache, v_cache, seq_lens, block_table, &a,
+                                &nothing);
+  if (rc != KVD_OK || nothing) return rc;
+  a.cow_src = cow_src;
+  return run_append(p, a, stream);
+}
+
 int kv_append_rope_shard(const kvd_params* p, void* q, const void* k_new, const void* v_new,
                          void* k_cache, void* v_cache, const int32_t* seq_lens,
                          const int32_t* shard_start, const int32_t* block_table, void* stream) {

@@ -35,6 +35,10 @@ struct AppendArgs {
   // Sequence-sharded mode: k and v of position p go to local slot
   // p - shard_start[b] (null: slot p); null caches rotate q only.
   const int32_t* shard_start;
+  // Copy on write of shared boundary pages (paged only): before its new
+  // tokens land, sequence b with cow_src[b] >= 0 gets slots 0 .. L_b % P - 1
+  // of page cow_src[b] copied into page block_table[b][L_b / P].
+  const int32_t* cow_src;
 };
 
 struct DecodeArgs {

@@ -62,6 +62,7 @@ class Workload:
     peaked_scale: float = 4.0
     cache_mode: str = "random"      # "random": draw stored cache; "prefill": draw raw prefix tokens
     config_id: int = 0
+    shared_prefix: int = 0          # paged: tokens (whole pages) every sequence shares
 
     @property
     def scale(self) -> float:
@@ -99,6 +100,10 @@ WORKLOADS = {
                            config_id=4),
     "long_ctx": Workload("long_ctx", 4, 32, 8, 128, "bf16", False, 1, 131072,
                          peaked_frac=0.01, peaked_scale=4.0, config_id=5),
+    # shared-prefix pages (prefix cache): 64 sequences over one 8192-token
+    # prefix held once in the pool, each with a private suffix of 16..1024 tokens
+    "shared_prefix": Workload("shared_prefix", 64, 64, 8, 128, "bf16", True, 1, None,
+                              len_range=(16, 1024), shared_prefix=8192, config_id=6),
 }
 
 
@@ -113,7 +118,26 @@ def draw_lengths(w: Workload, gen: torch.Generator) -> torch.Tensor:
     lo, hi = w.len_range
     u = torch.rand(w.batch, generator=gen, dtype=torch.float64)
     lens = torch.floor(torch.exp(math.log(lo) + u * (math.log(hi) - math.log(lo))))
-    return lens.clamp(lo, hi).to(torch.int64)
+    return lens.clamp(lo, hi).to(torch.int64) + w.shared_prefix
+
+
+def page_table(w: Workload, lens, gen: torch.Generator):
+    """Block table of a paged workload: each sequence's pages are consecutive
+    slices of one seeded permutation of the pool; with a shared prefix the
+    first shared_prefix / P entries of every row are the same pages.
+    Returns (block_table int32 [B, max_pages], num_pages)."""
+    P, T = w.page_size, w.q_len
+    n_sh = w.shared_prefix // P
+    own = [(int(L) + T + P - 1) // P - n_sh for L in lens]
+    num_pages = n_sh + sum(own)
+    perm = torch.randperm(num_pages, generator=gen).to(torch.int32)
+    bt = torch.full((w.batch, n_sh + max(own)), -1, dtype=torch.int32)
+    off = n_sh
+    for b, n in enumerate(own):
+        bt[b, :n_sh] = perm[:n_sh]
+        bt[b, n_sh:n_sh + n] = perm[off:off + n]
+        off += n
+    return bt, num_pages
 
 
 def _draw(shape, w: Workload, gen: torch.Generator) -> torch.Tensor:
@@ -150,20 +174,12 @@ def make_inputs(w: Workload, seed: int, fill: str = "nan") -> dict:
     P = w.page_size
 
     if w.paged:
-        pages_per_seq = [(int(L) + T + P - 1) // P for L in lens]
-        num_pages = sum(pages_per_seq)
-        max_pages = max(pages_per_seq)
-        perm = torch.randperm(num_pages, generator=gen).to(torch.int32)
-        bt = torch.full((B, max_pages), -1, dtype=torch.int32)
-        off = 0
-        for b, n in enumerate(pages_per_seq):
-            bt[b, :n] = perm[off:off + n]
-            off += n
+        bt, num_pages = page_table(w, lens, gen)
         k_cache = torch.full((num_pages, Hkv, P, D), fv, dtype=dt)
         v_cache = torch.full((num_pages, Hkv, P, D), fv, dtype=dt)
         out["block_table"] = bt
         out["num_pages"] = num_pages
-        out["max_pages_per_seq"] = max_pages
+        out["max_pages_per_seq"] = bt.shape[1]
     else:
         cap = round_up(int(lens.max()) + T, 16)
         k_cache = torch.full((B, Hkv, cap, D), fv, dtype=dt)
@@ -179,9 +195,10 @@ def make_inputs(w: Workload, seed: int, fill: str = "nan") -> dict:
     else:
         for b in range(B):
             L = int(lens[b])
+            t_lo = w.shared_prefix if b > 0 else 0   # the shared prefix is drawn once
             for h in range(Hkv):
-                k = _draw((L, D), w, gen)
-                v = _draw((L, D), w, gen)
+                k = _draw((L - t_lo, D), w, gen)
+                v = _draw((L - t_lo, D), w, gen)
                 if w.peaked_frac > 0:
                     n_peak = int(math.floor(w.peaked_frac * L))
                     idx = torch.randperm(L, generator=gen)[:n_peak]
@@ -189,7 +206,7 @@ def make_inputs(w: Workload, seed: int, fill: str = "nan") -> dict:
                 k = k.to(dt)
                 v = v.to(dt)
                 if w.paged:
-                    t = torch.arange(L)
+                    t = torch.arange(t_lo, L)
                     pages = out["block_table"][b, t // P].long()
                     k_cache[pages, h, t % P] = k
                     v_cache[pages, h, t % P] = v
@@ -239,14 +256,7 @@ def make_inputs_device(w: Workload, seed: int, device="cuda") -> dict:
     out["v_new"] = draw((B, T, Hkv, D)).to(dt)
     P = w.page_size
     if w.paged:
-        pages_per_seq = [(int(L) + T + P - 1) // P for L in lens]
-        num_pages = sum(pages_per_seq)
-        perm = torch.randperm(num_pages, generator=hgen).to(torch.int32)
-        bt = torch.full((B, max(pages_per_seq)), -1, dtype=torch.int32)
-        off = 0
-        for b, n in enumerate(pages_per_seq):
-            bt[b, :n] = perm[off:off + n]
-            off += n
+        bt, num_pages = page_table(w, lens, hgen)
         k_cache = torch.zeros((num_pages, Hkv, P, D), dtype=dt, device=device)
         v_cache = torch.zeros_like(k_cache)
         out.update(block_table=bt.to(device), num_pages=num_pages, max_pages_per_seq=bt.shape[1])
@@ -257,15 +267,16 @@ def make_inputs_device(w: Workload, seed: int, device="cuda") -> dict:
         out.update(block_table=None, max_seq_len=cap)
     for b in range(B):
         L = int(lens[b])
+        t_lo = w.shared_prefix if b > 0 else 0   # the shared prefix is drawn once
         for h in range(Hkv):
-            k = draw((L, D))
-            v = draw((L, D))
+            k = draw((L - t_lo, D))
+            v = draw((L - t_lo, D))
             if w.peaked_frac > 0:
                 n_peak = int(math.floor(w.peaked_frac * L))
                 idx = torch.randperm(L, generator=dgen, device=device)[:n_peak]
                 k[idx] *= w.peaked_scale
             if w.paged:
-                t = torch.arange(L, device=device)
+                t = torch.arange(t_lo, L, device=device)
                 pages = out["block_table"][b, t // P].long()
                 k_cache[pages, h, t % P] = k.to(dt)
                 v_cache[pages, h, t % P] = v.to(dt)
@@ -284,7 +295,11 @@ def step_bytes(w: Workload, seq_lens, out_esize: int) -> dict:
     written to the cache, the length (and page) indices read."""
     lens = [int(x) for x in seq_lens]
     B, T, Hq, Hkv, D, es = w.batch, w.q_len, w.num_heads, w.num_kv_heads, w.head_dim, w.esize
-    kv = sum(L + T for L in lens) * Hkv * 2 * D * es
+    # a shared prefix is stored once: its rows count once (the repeated reads
+    # of it by every sequence are cache hits, not HBM traffic the method needs)
+    sp = w.shared_prefix
+    kv = (sp + sum(L + T - sp for L in lens)) * Hkv * 2 * D * es
+    kv_logical = sum(L + T for L in lens) * Hkv * 2 * D * es
     q = B * T * Hq * D * es
     out = B * T * Hq * D * out_esize
     idx = B * 4
@@ -292,4 +307,5 @@ def step_bytes(w: Workload, seq_lens, out_esize: int) -> dict:
         idx += sum((L + T + w.page_size - 1) // w.page_size for L in lens) * 4
     decode = kv + q + out + idx
     append = 2 * q + 4 * B * T * Hkv * D * es + B * 4 + (B * T * 4 if w.paged else 0)
-    return {"decode": decode, "append": append, "step": decode + append, "kv": kv}
+    return {"decode": decode, "append": append, "step": decode + append, "kv": kv,
+            "kv_logical": kv_logical}

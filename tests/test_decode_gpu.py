@@ -55,6 +55,7 @@ SHAPES = {
                                                   cache_len=300),
     "tc_rows18_paged": WORKLOADS["paged_cb"].with_(batch=3, num_heads=12, num_kv_heads=2, q_len=3,
                                                    len_range=(1, 900)),
+    "shared_prefix": WORKLOADS["shared_prefix"].with_(batch=6, len_range=(1, 300), shared_prefix=512),
 }
 
 
