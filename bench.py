@@ -46,6 +46,9 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="CPU time budget of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cascade", action="store_true",
+                    help="shared_prefix workload: decode as prefix-once-per-group + suffix + merge "
+                         "(kv_cache_decode_rope_b200.prefix.cascade_decode)")
     ap.add_argument("--shard-seq", action="store_true",
                     help="sequence-sharded decode: every rank holds 1/N of each sequence's "
                          "positions; append + shard attention + all-gather of (o, lse) + merge "
@@ -238,7 +241,15 @@ def run_ours(args, rank, world, local):
         kvd.append_rope(q, kn, vn, inp["k_cache"], inp["v_cache"], seq, bt, rope_base=w.rope_base,
                         status=status)
 
+    if args.cascade and not w.shared_prefix:
+        raise SystemExit("--cascade needs a workload with a shared prefix")
+
     def decode(q, seq):
+        if args.cascade:
+            from kv_cache_decode_rope_b200.prefix import cascade_decode
+            cascade_decode(q, inp["k_cache"], inp["v_cache"], seq, bt, w.shared_prefix,
+                           scale=w.scale, out=out)
+            return
         if bt is None:
             kvd.decode_attention(q, inp["k_cache"], inp["v_cache"], seq, out, scale=w.scale,
                                  max_kv_len=mkl, workspace=ws, status=status)
@@ -359,7 +370,11 @@ def run_ours(args, rank, world, local):
         if dbt is not None:
             dbt.copy_(hbt, non_blocking=True)
         kvd.append_rope(dq, dk, dv, inp["k_cache"], inp["v_cache"], ds, dbt, rope_base=w.rope_base)
-        if dbt is None:
+        if args.cascade:
+            from kv_cache_decode_rope_b200.prefix import cascade_decode
+            cascade_decode(dq, inp["k_cache"], inp["v_cache"], ds, dbt, w.shared_prefix, scale=w.scale,
+                           out=out)
+        elif dbt is None:
             kvd.decode_attention(dq, inp["k_cache"], inp["v_cache"], ds, out, scale=w.scale,
                                  max_kv_len=mkl, workspace=ws)
         else:
@@ -497,7 +512,9 @@ def main():
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
             "l2": ("flushed between steps" if r["flush"] else
                    f"inputs larger than L2 ({r['cache_bytes'] / 2**20:.0f} MiB KV cache)"),
-            "step": "kv_append_rope + decode_attention" + ("_paged" if w.paged else ""),
+            "step": "kv_append_rope + " + ("cascade decode (prefix per group + suffix + merge)"
+                                           if args.cascade else
+                                           "decode_attention" + ("_paged" if w.paged else "")),
             "launch": "CUDA graph replay of the two library calls" if args.launch == "graph" else "eager calls",
             "max_kv_len": r["mkl"]}),
         "roofline": {
@@ -516,7 +533,7 @@ def main():
         "e2e": {"value": round(world * step_bytes / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
                 "us_per_step": round(e2e_ms * 1e3, 2),
                 "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
-        "gpu_launches": 3 * K,
+        "gpu_launches": (6 if args.cascade else 3) * K,
         "clocks": r["clocks"],
     }
     if args.driver_layers > 0:

@@ -99,3 +99,30 @@ def test_shared_prefix_decode(Hq, Hkv):
     err = oracle.max_abs_diff(np64(out), ref)
     log_error(f"shared_prefix[{Hq}/{Hkv}]", err)
     assert err <= 2e-3
+
+
+@pytest.mark.parametrize("dtype,Hq,Hkv,T,B", [(torch.bfloat16, 64, 8, 1, 12), (torch.float32, 8, 2, 2, 6),
+                                               (torch.bfloat16, 32, 8, 3, 8)])
+def test_cascade_decode_matches_plain_and_oracle(dtype, Hq, Hkv, T, B):
+    """Prefix once per group of sequences + suffix per sequence + merge equals
+    the plain paged decode and the oracle."""
+    from kv_cache_decode_rope_b200.prefix import cascade_decode
+    gen = torch.Generator().manual_seed(13)
+    D = 128 if dtype == torch.bfloat16 else 64
+    P, prefix = 16, 1024
+    priv = [int(x) for x in torch.randint(1, 12, (B,), generator=gen)]
+    k, v, bt, _ = _shared_pool(B, Hkv, D, P, prefix, priv, dtype, gen)
+    # lengths: the prefix plus up to the private capacity (a few tokens short of it)
+    seq = torch.tensor([prefix + 16 * n - T - (b % 3) for b, n in enumerate(priv)], dtype=torch.int32)
+    q = torch.randn((B, T, Hq, D), generator=gen).to(dtype)
+    dq, dk, dv, dbt, dseq = q.cuda(), k.cuda(), v.cuda(), bt.cuda(), seq.cuda()
+    got = cascade_decode(dq, dk, dv, dseq, dbt, prefix, scale=D ** -0.5, out_dtype=torch.float32)
+    plain = kvd.decode_attention_paged(dq, dk, dv, dseq, dbt, scale=D ** -0.5,
+                                       max_kv_len=int(seq.max()) + T, out_dtype=torch.float32)
+    ref = oracle.decode_attention(np64(q), np64(k), np64(v), seq.numpy(), D ** -0.5, bt.numpy())
+    torch.cuda.synchronize()
+    err = oracle.max_abs_diff(np64(got), ref)
+    log_error(f"cascade[{Hq}/{Hkv},T{T},B{B}]", err)
+    tol = 1e-5 if dtype == torch.float32 else 2e-3
+    assert err <= tol
+    assert oracle.max_abs_diff(np64(got), np64(plain)) <= tol
