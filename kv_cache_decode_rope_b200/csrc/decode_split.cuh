@@ -126,8 +126,10 @@ __device__ __forceinline__ int unit_chunks(int Nb) { return max(1, (Nb + kChunk 
 //
 // Block-wide exclusive scan of weighted chunks per sequence: sPrefix[b] = sum
 // over b' < b of (max(1, ceil(N_b' / 16)) + seg_cost), sPrefix[B] = total.  All threads of the block
-// call it; `scratch` holds one int per warp.  Ends with __syncthreads.
-__device__ __forceinline__ void chunk_prefix_scan(const DecodeArgs& a, int* sPrefix, int* scratch) {
+// call it; `scratch` holds one int per warp; `flag`: report lengths beyond
+// the capacity in the status word.  Ends with __syncthreads.
+__device__ __forceinline__ void chunk_prefix_scan(const DecodeArgs& a, int* sPrefix, int* scratch,
+                                                  bool flag) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nthr = blockDim.x;
   const int per = (a.B + nthr - 1) / nthr;
@@ -135,7 +137,7 @@ __device__ __forceinline__ void chunk_prefix_scan(const DecodeArgs& a, int* sPre
   const int hi = min(a.B, lo + per);
   int tsum = 0;
   for (int b = lo; b < hi; ++b)
-    tsum += unit_chunks(attended_len(a, b, blockIdx.x == 0)) + a.seg_cost;
+    tsum += unit_chunks(attended_len(a, b, flag)) + a.seg_cost;
   int incl = tsum;
 #pragma unroll
   for (int m = 1; m < 32; m <<= 1) {
@@ -246,7 +248,7 @@ __global__ void __launch_bounds__(NTW == 1 ? 288 : 160)
       mbar_init(&empty[s], ncw);
     }
   }
-  chunk_prefix_scan(a, sPrefix, reinterpret_cast<int*>(sML));  // sML is free until the first segment ends
+  chunk_prefix_scan(a, sPrefix, reinterpret_cast<int*>(sML), blockIdx.x == 0);  // sML is free until the first segment ends
   fence_barrier_init();
   fence_proxy_async_smem();
   __syncthreads();
@@ -254,7 +256,6 @@ __global__ void __launch_bounds__(NTW == 1 ? 288 : 160)
   grid_dep_launch();
 
   const long long total = (long long)a.Hkv * sPrefix[a.B];
-  if (blockIdx.x == 0 && threadIdx.x == 0) *a.total_chunks = total;
   const long long x0 = total * blockIdx.x / a.grid;
   const long long x1 = total * (blockIdx.x + 1) / a.grid;
   if (x0 >= x1) return;  // empty range: no copies issued, nothing to write
@@ -610,21 +611,28 @@ __global__ void __launch_bounds__(NTW == 1 ? 288 : 160)
         if (d == 0) a.part_lse[(size_t)slot_idx * a.R + rglob] = (L > 0.f) ? Ms + fast_log2(L) : -INFINITY;
       }
     }
-    if (threadIdx.x == 0) {
-      if (sg.k0 == 0) a.unit_ctas[u].x = blockIdx.x;
-      if (sg.kend == sg.nb) a.unit_ctas[u].y = blockIdx.x;
-    }
     named_bar_sync(1, ncons);
   }
 }
 
+// CTA holding global weighted chunk x of a split over `total` chunks: the
+// largest c with floor(total c / grid) <= x.
+__device__ __forceinline__ int cta_of_chunk(long long x, long long total, int grid) {
+  return (int)(((x + 1) * grid - 1) / total);
+}
+
 // Kernel C: one warp per (unit, row) merges the partials of units split over
 // several CTAs: out = sum_s 2^(lse_s - LSE) o_s with LSE = log2 sum_s 2^lse_s.
-// Lane j fetches the log-sum-exp of partials j, j + 32, ...; each lane then
-// reads its D / 32 dimensions of four partial rows at a time, so the merge
-// costs a handful of dependent memory round trips whatever the split count.
+// The CTAs that share a unit follow from the split itself, which every block
+// recomputes from the sequence lengths before the decode kernel finishes, so
+// after the wait only the partials are read: lane j fetches the log-sum-exp
+// of partial j while every lane fetches its D / 32 dimensions of the first
+// four partial rows, all in one round trip; longer splits continue four
+// partial rows at a time.
 template <int D>
 __global__ void __launch_bounds__(256) combine_kernel(DecodeArgs a) {
+  extern __shared__ int sPrefix[];   // [B + 1] chunk prefix, then one int per warp
+  chunk_prefix_scan(a, sPrefix, sPrefix + a.B + 1, false);
   grid_dep_wait();      // the partials of the decode kernel
   grid_dep_launch();
   constexpr int PER = D >= 32 ? D / 32 : 1;   // dimensions per lane
@@ -635,70 +643,85 @@ __global__ void __launch_bounds__(256) combine_kernel(DecodeArgs a) {
   if (wid >= U * a.R) return;
   const int u = (int)(wid / a.R);
   const int r = (int)(wid % a.R);
-  const int2 cr = a.unit_ctas[u];
-  const long long total = *a.total_chunks;
-  if (cr.x >= cr.y) return;  // one CTA covered the unit and wrote out directly
-  const int n = cr.y - cr.x + 1;
+  const int b = u / a.Hkv, hk = u % a.Hkv;
+  // the unit's real chunks in the weighted index space, and their CTAs
+  const long long total = (long long)a.Hkv * sPrefix[a.B];
+  const int ext = sPrefix[b + 1] - sPrefix[b];
+  const long long first = (long long)a.Hkv * sPrefix[b] + (long long)hk * ext + a.seg_cost;
+  const long long last = (long long)a.Hkv * sPrefix[b] + (long long)(hk + 1) * ext - 1;
+  const int c0 = cta_of_chunk(first, total, a.grid);
+  const int c1 = cta_of_chunk(last, total, a.grid);
+  if (c0 >= c1) return;  // one CTA covered the unit and wrote out directly
+  const int n = c1 - c0 + 1;
   // CTAs whose chunk range came out empty wrote no partial: weight 0
+  const bool all_full = total >= a.grid;
   auto lse_of = [&](int j) -> float {
-    const int c = cr.x + j;
-    if (total * c / a.grid >= total * (c + 1) / a.grid) return -INFINITY;
+    const int c = c0 + j;
+    if (!all_full && total * c / a.grid >= total * (c + 1) / a.grid) return -INFINITY;
     return a.part_lse[((size_t)c + u) * a.R + r];
   };
-  float M = -INFINITY;
-  for (int j = lane; j < n; j += 32) M = fmaxf(M, lse_of(j));
+
+  const size_t stride = (size_t)a.R * D;  // between the partial rows of consecutive CTAs
+  const float* base = a.part_o + ((size_t)(c0 + u) * a.R + r) * D + (size_t)lane * PER;
+  auto load_row = [&](int j, float* x) {
+    const float* src = base + (size_t)j * stride;
+    if (lane < LANES) {
+      if constexpr (PER % 4 == 0) {
+#pragma unroll
+        for (int e = 0; e < PER; e += 4) {
+          const float4 v = *reinterpret_cast<const float4*>(src + e);
+          x[e] = v.x; x[e + 1] = v.y; x[e + 2] = v.z; x[e + 3] = v.w;
+        }
+      } else if constexpr (PER == 2) {
+        const float2 v = *reinterpret_cast<const float2*>(src);
+        x[0] = v.x; x[1] = v.y;
+      } else {
+        x[0] = src[0];
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < PER; ++e) x[e] = 0.f;
+    }
+  };
+  // first round trip: the first (up to) four partial rows and every partial's lse
+  float x[4][PER];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) load_row(min(i, n - 1), x[i]);
+  const int nl = (n + 31) / 32;   // lse values per lane
+  // lse of partial lane (kept: the weights of the first 32 partials need no reload)
+  const float l0 = (lane < n) ? lse_of(lane) : -INFINITY;
+  float M = l0;
+  for (int t = 1; t < nl; ++t)
+    if (t * 32 + lane < n) M = fmaxf(M, lse_of(t * 32 + lane));
 #pragma unroll
   for (int m = 16; m >= 1; m >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, m));
   const float Ms = (M == -INFINITY) ? 0.f : M;
-
-  const size_t stride = (size_t)a.R * D;  // between the partial rows of consecutive CTAs
-  const float* base = a.part_o + ((size_t)(cr.x + u) * a.R + r) * D + (size_t)lane * PER;
+  float L = 0.f;
   float acc[PER];
 #pragma unroll
   for (int e = 0; e < PER; ++e) acc[e] = 0.f;
-  float L = 0.f;
-  for (int j0 = 0; j0 < n; j0 += 32) {
-    const float lj = (j0 + lane < n) ? lse_of(j0 + lane) : -INFINITY;
-    const float w = (lj == -INFINITY) ? 0.f : fast_exp2(lj - Ms);
+  for (int t = 0; t < nl; ++t) {
+    const float lt = (t == 0) ? l0 : (t * 32 + lane < n) ? lse_of(t * 32 + lane) : -INFINITY;
+    const float w = (lt == -INFINITY) ? 0.f : fast_exp2(lt - Ms);
     L += w;
-    const int m = min(32, n - j0);
+    const int m = min(32, n - t * 32);
     for (int k = 0; k < m; k += 4) {
-      float wk[4];
-      float x[4][PER];
+      if (t > 0 || k > 0) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int kk = min(k + i, m - 1);             // past the end: reload a valid row, weight 0
-        wk[i] = __shfl_sync(0xffffffffu, w, kk);
-        if (k + i >= m) wk[i] = 0.f;
-        const float* src = base + (size_t)(j0 + kk) * stride;
-        if (lane < LANES) {
-          if constexpr (PER % 4 == 0) {
-#pragma unroll
-            for (int e = 0; e < PER; e += 4) {
-              const float4 v = *reinterpret_cast<const float4*>(src + e);
-              x[i][e] = v.x; x[i][e + 1] = v.y; x[i][e + 2] = v.z; x[i][e + 3] = v.w;
-            }
-          } else if constexpr (PER == 2) {
-            const float2 v = *reinterpret_cast<const float2*>(src);
-            x[i][0] = v.x; x[i][1] = v.y;
-          } else {
-            x[i][0] = src[0];
-          }
-        } else {
-#pragma unroll
-          for (int e = 0; e < PER; ++e) x[i][e] = 0.f;
-        }
+        for (int i = 0; i < 4; ++i) load_row(t * 32 + min(k + i, m - 1), x[i]);
       }
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
+      for (int i = 0; i < 4; ++i) {
+        float wk = __shfl_sync(0xffffffffu, w, min(k + i, m - 1));
+        if (k + i >= m) wk = 0.f;   // past the end: a valid row reloaded, weight 0
 #pragma unroll
-        for (int e = 0; e < PER; ++e) acc[e] += (wk[i] != 0.f) ? wk[i] * x[i][e] : 0.f;
+        for (int e = 0; e < PER; ++e) acc[e] += (wk != 0.f) ? wk * x[i][e] : 0.f;
+      }
     }
   }
 #pragma unroll
   for (int m = 16; m >= 1; m >>= 1) L += __shfl_xor_sync(0xffffffffu, L, m);
   if (lane >= LANES) return;
-  const int b = u / a.Hkv, hk = u % a.Hkv;
   const int i = r / a.g;
   const int h = hk * a.g + r % a.g;
   const size_t orow = ((size_t)b * a.T + i) * a.Hq + h;
@@ -734,6 +757,10 @@ __global__ void __launch_bounds__(256) combine_kernel(DecodeArgs a) {
   }
 }
 
+// Dynamic shared memory of the merge kernel: the chunk prefix and the scan's
+// per-warp scratch.
+inline size_t combine_smem(int B) { return (size_t)(B + 1 + 8) * sizeof(int); }
+
 // ---------------------------------------------------------------- host side
 inline int d_index(int D) {
   return D == 16 ? 0 : D == 32 ? 1 : D == 64 ? 2 : D == 128 ? 3 : D == 256 ? 4 : -1;
@@ -767,7 +794,7 @@ cudaError_t launch_one(const DecodeArgs& a, int nrg, int cfg_idx, cudaStream_t s
   if (e != cudaSuccess) return e;
   const long long warps = (long long)a.B * a.Hkv * a.R;
   const int cblocks = (int)((warps * 32 + 255) / 256);
-  return launch_pdl(combine_kernel<D>, dim3(cblocks), dim3(256), 0, st, a);
+  return launch_pdl(combine_kernel<D>, dim3(cblocks), dim3(256), combine_smem(a.B), st, a);
 }
 
 template <typename T, int D, bool PAGED>

@@ -226,7 +226,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   }
   if (warp == WARP_KLOAD && lane == 0) prefetch_tensormap(&tmk);
   if (warp == WARP_VLOAD && lane == 0) prefetch_tensormap(&tmv);
-  chunk_prefix_scan(a, sPrefix, sScratch);
+  chunk_prefix_scan(a, sPrefix, sScratch, blockIdx.x == 0);
   fence_barrier_init();
   fence_proxy_async_smem();
   tc_fence_before();
@@ -237,7 +237,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   grid_dep_launch();
 
   const long long total = (long long)a.Hkv * sPrefix[a.B];
-  if (blockIdx.x == 0 && threadIdx.x == 0) *a.total_chunks = total;
   const long long x0 = total * blockIdx.x / a.grid;
   const long long x1 = total * (blockIdx.x + 1) / a.grid;
 
@@ -661,10 +660,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           if (!whole) a.part_lse[(size_t)slot_idx * a.R + qr] = lse;
           else if (a.out_lse) a.out_lse[ob / TC_D] = lse;
         }
-        if (threadIdx.x == 0) {
-          if (sg.k0 == 0) a.unit_ctas[u].x = blockIdx.x;
-          if (sg.kend == sg.nb) a.unit_ctas[u].y = blockIdx.x;
-        }
         tc_fence_before();  // the O reads above precede the next segment's first PV
         named_bar_sync(1, TC_SOFTMAX_THREADS);   // sML is reused by the next segment
 
@@ -732,7 +727,8 @@ cudaError_t launch_tc(const DecodeArgs& a, cudaStream_t st) {
   e = launch_pdl(decode_tc_kernel<PAGED, M>, dim3(a.grid), dim3(TC_THREADS), smem, st, a, mk, mv);
   if (e != cudaSuccess) return e;
   const long long warps = (long long)a.B * a.Hkv * a.R;
-  return launch_pdl(combine_kernel<TC_D>, dim3((int)((warps * 32 + 255) / 256)), dim3(256), 0, st, a);
+  return launch_pdl(combine_kernel<TC_D>, dim3((int)((warps * 32 + 255) / 256)), dim3(256),
+                    combine_smem(a.B), st, a);
 }
 
 }  // namespace

@@ -104,8 +104,6 @@ int prepare_decode(const kvd_params* p, const void* q, const void* k_cache, cons
   a.out = out;
   a.part_o = reinterpret_cast<float*>(ws + wl.part_o_off);
   a.part_lse = reinterpret_cast<float*>(ws + wl.part_lse_off);
-  a.unit_ctas = reinterpret_cast<int2*>(ws + wl.unit_ctas_off);
-  a.total_chunks = reinterpret_cast<long long*>(ws + wl.total_off);
   a.status = p->status;
   a.B = p->batch;
   a.T = p->q_len;
@@ -212,9 +210,7 @@ WorkspaceLayout workspace_layout(int B, int Hkv, int R, int D) {
   WorkspaceLayout w{};
   const size_t U = (size_t)B * Hkv;
   const size_t slots = (size_t)kMaxGrid + U;
-  w.unit_ctas_off = 0;
-  w.total_off = align_up(U * sizeof(int2));
-  w.part_lse_off = w.total_off + kAlign;
+  w.part_lse_off = 0;
   w.part_o_off = align_up(w.part_lse_off + slots * R * sizeof(float));
   w.total = align_up(w.part_o_off + slots * R * D * sizeof(float));
   return w;

@@ -50,8 +50,6 @@ struct DecodeArgs {
   void* out;
   float* part_o;      // [slots, R, D]
   float* part_lse;    // [slots, R]
-  int2* unit_ctas;    // [U]: first and last CTA that touched each (sequence, kv head)
-  long long* total_chunks;  // written by CTA 0: length of the weighted chunk space (defines every CTA's range)
   int* status;
   int B, T, Hq, Hkv, g, R, D;
   int max_seq_len;                       // contiguous capacity
@@ -81,7 +79,7 @@ cudaError_t launch_merge_shards(const MergeArgs& a, cudaStream_t st);
 
 // Workspace carve-up, shared by kvd_workspace_size and the launch.
 struct WorkspaceLayout {
-  size_t unit_ctas_off, total_off, part_lse_off, part_o_off, total;
+  size_t part_lse_off, part_o_off, total;
 };
 WorkspaceLayout workspace_layout(int B, int Hkv, int R, int D);
 

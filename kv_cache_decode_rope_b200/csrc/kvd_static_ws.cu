@@ -98,9 +98,7 @@ extern "C" int decode_attention_static(const kvd_params* p, const void* q, const
                              p->dtype == KVD_BF16, (int)R);
   const size_t U = (size_t)p->batch * p->num_kv_heads;
   const size_t slots = (size_t)grid + U;
-  const size_t unit_off = 0;
-  const size_t total_off = align256(U * sizeof(int2));
-  const size_t lse_off = total_off + 256;
+  const size_t lse_off = 0;
   const size_t o_off = align256(lse_off + slots * (size_t)R * sizeof(float));
   const size_t need = align256(o_off + slots * (size_t)R * p->head_dim * sizeof(float));
   if (need > (size_t)KVD_STATIC_WORKSPACE_BYTES) return KVD_ERR_WORKSPACE;
@@ -115,8 +113,6 @@ extern "C" int decode_attention_static(const kvd_params* p, const void* q, const
   a.out = out;
   a.part_o = reinterpret_cast<float*>(ws + o_off);
   a.part_lse = reinterpret_cast<float*>(ws + lse_off);
-  a.unit_ctas = reinterpret_cast<int2*>(ws + unit_off);
-  a.total_chunks = reinterpret_cast<long long*>(ws + total_off);
   a.status = p->status;
   a.B = p->batch;
   a.T = p->q_len;
