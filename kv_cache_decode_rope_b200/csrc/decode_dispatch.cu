@@ -34,10 +34,12 @@ int decode_grid(int B, int Hkv, int max_kv_len, int num_sms, int D, int bf16, in
 }
 
 // Virtual chunks charged per unit in the work split (the cost of a unit
-// boundary, in 16-token chunks of streaming): about two 128-token stages for
-// the tensor-core kernel (epilogue, pipeline refill), half that for the
-// CUDA-core kernel, whose CTAs each stream at half an SM's bandwidth.
-constexpr int kSegCostTc = 16;
+// boundary, in 16-token chunks of streaming): about four 128-token stages for
+// the tensor-core kernel (q load, pipeline drain and refill, epilogue; a sweep
+// of 16..64 on the MTP-verify and continuous-batching workloads put the best
+// at 32-40), 8 for the CUDA-core kernel, whose CTAs each stream at half an
+// SM's bandwidth.
+constexpr int kSegCostTc = 32;
 constexpr int kSegCostCore = 8;
 
 cudaError_t launch_decode(const DecodeArgs& args, int bf16, cudaStream_t st) {
