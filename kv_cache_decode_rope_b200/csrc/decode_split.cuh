@@ -73,9 +73,15 @@ struct Smem {
   __host__ __device__ static size_t p_off() { return bars_off() + 2 * G::NSTAGES * 8; }
   __host__ __device__ static size_t comb_off(int ncw) { return p_off() + (size_t)ncw * P_FLOATS * 4; }
   __host__ __device__ static size_t ml_off(int ncw) { return comb_off(ncw) + (size_t)ncw * RPW * D * 4; }
-  __host__ __device__ static size_t prefix_off(int ncw) { return ml_off(ncw) + (size_t)ncw * RPW * 2 * 4; }
-  __host__ __device__ static size_t total(int ncw, int B) {
-    return prefix_off(ncw) + (size_t)(B + 1) * 4;
+  // one group's region (stage rings to merge scratch), 1 KB aligned
+  __host__ __device__ static size_t group_bytes(int ncw) {
+    return (ml_off(ncw) + (size_t)ncw * RPW * 2 * 4 + 1023) / 1024 * 1024;
+  }
+  // after the groups: the per-sequence chunk prefix [B + 1], then one int per
+  // warp of the block for its scan
+  __host__ __device__ static size_t prefix_off(int ncw, int groups) { return groups * group_bytes(ncw); }
+  __host__ __device__ static size_t total(int ncw, int B, int groups) {
+    return prefix_off(ncw, groups) + (size_t)(B + 1 + 32) * 4;
   }
 };
 
@@ -205,8 +211,13 @@ __device__ __forceinline__ bool next_has_work(const DecodeArgs& a, const Seg& s,
   return x1 - s.next_x > a.seg_cost;
 }
 
-template <typename T, int D, int RPW, int NTW, bool PAGED>
-__global__ void __launch_bounds__(NTW == 1 ? 288 : 160)
+// GROUPS = 2: one block holds two independent producer + consumer groups,
+// each playing one CTA of the split (block b plays CTAs 2b and 2b + 1) with its
+// own rings, barriers and named barrier.  Two separate blocks on one SM do not
+// progress at the same rate (the one placed first is favoured and ends ~15%
+// earlier, leaving the SM half used for the rest); two groups of one block do.
+template <typename T, int D, int RPW, int NTW, bool PAGED, int GROUPS>
+__global__ void __launch_bounds__(GROUPS == 2 ? 320 : (NTW == 1 ? 288 : 160))
     decode_kernel(DecodeArgs a, int nrg) {
   using G = Geo<T, D>;
   using S = Smem<T, D, RPW, NTW>;
@@ -223,10 +234,16 @@ __global__ void __launch_bounds__(NTW == 1 ? 288 : 160)
   static_assert(NV * TPP * NBLK * NTW == RPW * G::STAGE_TOKENS, "block tiling");
   static_assert(NOWN <= RPW, "each lane's scores must belong to distinct rows");
 
-  extern __shared__ __align__(128) unsigned char smem[];
+  extern __shared__ __align__(1024) unsigned char smem_all[];
   const int ncw = nrg * NTW;                 // consumer warps
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
+  const int gthreads = (ncw + 1) * 32;       // threads of one group
+  const int grp = GROUPS == 2 ? (int)threadIdx.x / gthreads : 0;
+  const int tid = (int)threadIdx.x - grp * gthreads;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int vcta = (int)blockIdx.x * GROUPS + grp;   // the CTA of the split this group plays
+  const int bar = 1 + grp;                           // the group's named barrier
+  unsigned char* smem = smem_all + (size_t)grp * S::group_bytes(ncw);
   T* sK = reinterpret_cast<T*>(smem);
   T* sV = reinterpret_cast<T*>(smem + (size_t)G::NSTAGES * G::STAGE_BYTES);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::bars_off());
@@ -234,21 +251,21 @@ __global__ void __launch_bounds__(NTW == 1 ? 288 : 160)
   float* sP = reinterpret_cast<float*>(smem + S::p_off());
   float* sComb = reinterpret_cast<float*>(smem + S::comb_off(ncw));
   float* sML = reinterpret_cast<float*>(smem + S::ml_off(ncw));
-  int* sPrefix = reinterpret_cast<int*>(smem + S::prefix_off(ncw));
+  int* sPrefix = reinterpret_cast<int*>(smem_all + S::prefix_off(ncw, GROUPS));
 
   // ---- prologue: clear stages, barriers, per-sequence chunk prefix --------
   {
     uint4* z = reinterpret_cast<uint4*>(smem);
     const int n16 = (int)(S::stages() / 16);
-    for (int k = threadIdx.x; k < n16; k += blockDim.x) z[k] = make_uint4(0, 0, 0, 0);
+    for (int k = tid; k < n16; k += gthreads) z[k] = make_uint4(0, 0, 0, 0);
   }
-  if (threadIdx.x == 0) {
+  if (tid == 0) {
     for (int s = 0; s < G::NSTAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], ncw);
     }
   }
-  chunk_prefix_scan(a, sPrefix, reinterpret_cast<int*>(sML), blockIdx.x == 0);  // sML is free until the first segment ends
+  chunk_prefix_scan(a, sPrefix, sPrefix + a.B + 1, blockIdx.x == 0);
   fence_barrier_init();
   fence_proxy_async_smem();
   __syncthreads();
@@ -256,8 +273,9 @@ __global__ void __launch_bounds__(NTW == 1 ? 288 : 160)
   grid_dep_launch();
 
   const long long total = (long long)a.Hkv * sPrefix[a.B];
-  const long long x0 = total * blockIdx.x / a.grid;
-  const long long x1 = total * (blockIdx.x + 1) / a.grid;
+  if (vcta >= a.grid) return;  // the second group of an odd grid's last block
+  const long long x0 = total * vcta / a.grid;
+  const long long x1 = total * (vcta + 1) / a.grid;
   if (x0 >= x1) return;  // empty range: no copies issued, nothing to write
 
   const SegState st = locate_chunk(a, sPrefix, x0);
@@ -577,11 +595,11 @@ __global__ void __launch_bounds__(NTW == 1 ? 288 : 160)
 #pragma unroll
       for (int r = 0; r < RPW; ++r) sML[((size_t)warp * RPW + r) * 2] = m_all[r];
     }
-    named_bar_sync(1, ncons);
+    named_bar_sync(bar, ncons);
 
     const bool whole = sg.whole();
-    const long long slot_idx = (long long)blockIdx.x + u;
-    for (int e = threadIdx.x; e < nrg * RPW * D; e += ncons) {
+    const long long slot_idx = (long long)vcta + u;
+    for (int e = tid; e < nrg * RPW * D; e += ncons) {
       const int rgi = e / (RPW * D);
       const int r = (e / D) % RPW;
       const int d = e % D;
@@ -611,7 +629,7 @@ __global__ void __launch_bounds__(NTW == 1 ? 288 : 160)
         if (d == 0) a.part_lse[(size_t)slot_idx * a.R + rglob] = (L > 0.f) ? Ms + fast_log2(L) : -INFINITY;
       }
     }
-    named_bar_sync(1, ncons);
+    named_bar_sync(bar, ncons);
   }
 }
 
@@ -769,42 +787,55 @@ inline int d_index(int D) {
 // Per (D, row config): devices on which the shared-memory opt-in was set.
 template <typename T, bool PAGED>
 std::atomic<unsigned long long>& smem_attr_flag(int di, int cfg) {
-  static std::atomic<unsigned long long> flags[5][6];
+  static std::atomic<unsigned long long> flags[5][12];
   return flags[di][cfg];
 }
 
-template <typename T, int D, int RPW, int NTW, bool PAGED>
-cudaError_t launch_one(const DecodeArgs& a, int nrg, int cfg_idx, cudaStream_t st) {
+// One launch of the split kernel with `groups` CTAs of the split per block
+// (2 when the configuration is one of two CTAs per SM and both groups' shared
+// memory fits a block, else 1).
+template <typename T, int D, int RPW, int NTW, bool PAGED, int GROUPS>
+cudaError_t launch_groups(const DecodeArgs& a, int nrg, int cfg_idx, cudaStream_t st) {
   using S = Smem<T, D, RPW, NTW>;
   const int ncw = nrg * NTW;
-  const size_t smem = S::total(ncw, a.B);
+  const size_t smem = S::total(ncw, a.B, GROUPS);
   if (smem > 227 * 1024) return cudaErrorNotSupported;
-  auto kern = decode_kernel<T, D, RPW, NTW, PAGED>;
+  auto kern = decode_kernel<T, D, RPW, NTW, PAGED, GROUPS>;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  auto& flag = smem_attr_flag<T, PAGED>(d_index(D), cfg_idx);
+  auto& flag = smem_attr_flag<T, PAGED>(d_index(D), cfg_idx + (GROUPS == 2 ? 6 : 0));
   const unsigned long long bit = 1ull << (dev & 63);
   if (!(flag.load() & bit)) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
     if (e != cudaSuccess) return e;
     flag.fetch_or(bit);
   }
-  e = launch_pdl(kern, dim3(a.grid), dim3((ncw + 1) * 32), smem, st, a, nrg);
+  e = launch_pdl(kern, dim3((a.grid + GROUPS - 1) / GROUPS), dim3(GROUPS * (ncw + 1) * 32), smem,
+                 st, a, nrg);
   if (e != cudaSuccess) return e;
   const long long warps = (long long)a.B * a.Hkv * a.R;
   const int cblocks = (int)((warps * 32 + 255) / 256);
   return launch_pdl(combine_kernel<D>, dim3(cblocks), dim3(256), combine_smem(a.B), st, a);
 }
 
+// Configurations of up to 4 rows run two CTAs of the split per block while
+// both groups' shared memory fits (the per-sequence prefix grows with B).
+template <typename T, int D, int RPW, bool PAGED>
+cudaError_t launch_paired(const DecodeArgs& a, int cfg_idx, cudaStream_t st) {
+  const cudaError_t e = launch_groups<T, D, RPW, 4, PAGED, 2>(a, 1, cfg_idx, st);
+  if (e != cudaErrorNotSupported) return e;
+  return launch_groups<T, D, RPW, 4, PAGED, 1>(a, 1, cfg_idx, st);
+}
+
 template <typename T, int D, bool PAGED>
 cudaError_t launch_rows(const DecodeArgs& a, cudaStream_t st) {
-  if (a.R <= 1) return launch_one<T, D, 1, 4, PAGED>(a, 1, 0, st);
-  if (a.R <= 2) return launch_one<T, D, 2, 4, PAGED>(a, 1, 1, st);
-  if (a.R <= 4) return launch_one<T, D, 4, 4, PAGED>(a, 1, 2, st);
-  if (a.R <= 8) return launch_one<T, D, 8, 4, PAGED>(a, 1, 3, st);
-  if (a.R <= 16) return launch_one<T, D, 8, 2, PAGED>(a, 2, 4, st);
-  if (a.R <= kMaxRows) return launch_one<T, D, 8, 1, PAGED>(a, (a.R + 7) / 8, 5, st);
+  if (a.R <= 1) return launch_paired<T, D, 1, PAGED>(a, 0, st);
+  if (a.R <= 2) return launch_paired<T, D, 2, PAGED>(a, 1, st);
+  if (a.R <= 4) return launch_paired<T, D, 4, PAGED>(a, 2, st);
+  if (a.R <= 8) return launch_groups<T, D, 8, 4, PAGED, 1>(a, 1, 3, st);
+  if (a.R <= 16) return launch_groups<T, D, 8, 2, PAGED, 1>(a, 2, 4, st);
+  if (a.R <= kMaxRows) return launch_groups<T, D, 8, 1, PAGED, 1>(a, (a.R + 7) / 8, 5, st);
   return cudaErrorNotSupported;
 }
 
