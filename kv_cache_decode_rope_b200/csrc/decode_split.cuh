@@ -77,11 +77,11 @@ struct Smem {
   __host__ __device__ static size_t group_bytes(int ncw) {
     return (ml_off(ncw) + (size_t)ncw * RPW * 2 * 4 + 1023) / 1024 * 1024;
   }
-  // after the groups: the per-sequence chunk prefix [B + 1], then one int per
-  // warp of the block for its scan
+  // after the groups: the per-sequence chunk prefix [B + 1], one int per warp
+  // of the block for its scan, then N_b per sequence [B]
   __host__ __device__ static size_t prefix_off(int ncw, int groups) { return groups * group_bytes(ncw); }
   __host__ __device__ static size_t total(int ncw, int B, int groups) {
-    return prefix_off(ncw, groups) + (size_t)(B + 1 + 32) * 4;
+    return prefix_off(ncw, groups) + (size_t)(2 * B + 1 + 32) * 4;
   }
 };
 
@@ -133,9 +133,10 @@ __device__ __forceinline__ int unit_chunks(int Nb) { return max(1, (Nb + kChunk 
 // Block-wide exclusive scan of weighted chunks per sequence: sPrefix[b] = sum
 // over b' < b of (max(1, ceil(N_b' / 16)) + seg_cost), sPrefix[B] = total.  All threads of the block
 // call it; `scratch` holds one int per warp; `flag`: report lengths beyond
-// the capacity in the status word.  Ends with __syncthreads.
+// the capacity in the status word; `sNb` (optional): receives N_b per
+// sequence.  Ends with __syncthreads.
 __device__ __forceinline__ void chunk_prefix_scan(const DecodeArgs& a, int* sPrefix, int* scratch,
-                                                  bool flag) {
+                                                  bool flag, int* sNb = nullptr) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nthr = blockDim.x;
   const int per = (a.B + nthr - 1) / nthr;
@@ -157,7 +158,9 @@ __device__ __forceinline__ void chunk_prefix_scan(const DecodeArgs& a, int* sPre
   int run = woff + incl - tsum;
   for (int b = lo; b < hi; ++b) {
     sPrefix[b] = run;
-    run += unit_chunks(attended_len(a, b, false)) + a.seg_cost;
+    const int nb = attended_len(a, b, false);
+    if (sNb) sNb[b] = nb;
+    run += unit_chunks(nb) + a.seg_cost;
   }
   if (hi == a.B && lo < hi) sPrefix[a.B] = run;
   __syncthreads();
@@ -265,7 +268,8 @@ __global__ void __launch_bounds__(GROUPS == 2 ? 320 : (NTW == 1 ? 288 : 160))
       mbar_init(&empty[s], ncw);
     }
   }
-  chunk_prefix_scan(a, sPrefix, sPrefix + a.B + 1, blockIdx.x == 0);
+  int* sNb = sPrefix + a.B + 1 + 32;   // attended lengths, read once here
+  chunk_prefix_scan(a, sPrefix, sPrefix + a.B + 1, blockIdx.x == 0, sNb);
   fence_barrier_init();
   fence_proxy_async_smem();
   __syncthreads();
@@ -288,7 +292,7 @@ __global__ void __launch_bounds__(GROUPS == 2 ? 320 : (NTW == 1 ? 288 : 160))
     for (; p.x < x1 && !failed; next_unit(a, p, seg_of(a, sPrefix, p, x1))) {
       const Seg sg = seg_of(a, sPrefix, p, x1);
       if (sg.empty()) continue;
-      const int Nb = attended_len(a, p.b, false);
+      const int Nb = sNb[p.b];
       const int kend = sg.kend;
       // page ids of the sequence, two 32-chunk windows: the second is loaded
       // 32 chunks ahead of its use so the block-table latency stays off the issue path
@@ -385,13 +389,23 @@ __global__ void __launch_bounds__(GROUPS == 2 ? 320 : (NTW == 1 ? 288 : 160))
   for (int i = 0; i < NOWN; ++i) own_tok[i] = (i + NOWN * (lg >> SHIFT)) / RPW;
   float* myP = sP + warp * S::P_FLOATS;
 
+  // this lane's 16-byte slice of q row r of unit (b, hk) (null past the rows)
+  auto q_ptr = [&](int b, int hk, int r) -> const uint4* {
+    const int rglob = rg * RPW + r;
+    if (rglob >= a.R) return nullptr;
+    const int i = rglob / a.g;
+    const int h = hk * a.g + rglob % a.g;
+    return reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(a.q) +
+                                          (((size_t)b * a.T + i) * a.Hq + h) * D + lg * EPV);
+  };
+
   int s = 0;
   bool failed = false;
   SegState c = st;
   for (; c.x < x1; next_unit(a, c, seg_of(a, sPrefix, c, x1))) {
     const Seg sg = seg_of(a, sPrefix, c, x1);
     if (sg.empty()) continue;
-    const int Nb = attended_len(a, c.b, false);
+    const int Nb = sNb[c.b];
     const int Lb = mask_base(a, c.b, Nb);  // local position of the first new token (may be <= 0)
     const int kend = sg.kend;
     const int u = c.b * a.Hkv + c.hk;
@@ -404,20 +418,23 @@ __global__ void __launch_bounds__(GROUPS == 2 ? 320 : (NTW == 1 ? 288 : 160))
     int vis_own[NOWN];  // visible token count of own rows
 #pragma unroll
     for (int r = 0; r < RPW; ++r) {
-      const int rglob = rg * RPW + r;
       m_all[r] = -INFINITY;
+      const uint4* qp = q_ptr(c.b, c.hk, r);
+      const uint4 qv = qp ? *qp : make_uint4(0u, 0u, 0u, 0u);
+      float2 f[NP];
+      VT::unpack(qv, f);
 #pragma unroll
-      for (int e = 0; e < NP; ++e) { o2[r][e] = make_float2(0.f, 0.f); q2[r][e] = make_float2(0.f, 0.f); }
-      if (rglob < a.R) {
-        const int i = rglob / a.g;
-        const int h = c.hk * a.g + rglob % a.g;
-        const T* qp = reinterpret_cast<const T*>(a.q) + (((size_t)c.b * a.T + i) * a.Hq + h) * D + lg * EPV;
-        float2 f[NP];
-        VT::unpack(*reinterpret_cast<const uint4*>(qp), f);
-#pragma unroll
-        for (int e = 0; e < NP; ++e) q2[r][e] = make_float2(f[e].x * a.qscale, f[e].y * a.qscale);
+      for (int e = 0; e < NP; ++e) {
+        o2[r][e] = make_float2(0.f, 0.f);
+        q2[r][e] = make_float2(f[e].x * a.qscale, f[e].y * a.qscale);
       }
     }
+    // the unit after this one, if this slice reaches it: its q is prefetched
+    // into L1 during this segment's last stage, so that the load at the
+    // segment change does not wait on HBM under full load
+    const bool prefetch_next = next_has_work(a, sg, x1);
+    const int nx_hk = (c.hk + 1 == a.Hkv) ? 0 : c.hk + 1;
+    const int nx_b = (c.hk + 1 == a.Hkv) ? c.b + 1 : c.b;
 #pragma unroll
     for (int i = 0; i < NOWN; ++i) {
       m_own[i] = -INFINITY;
@@ -429,6 +446,13 @@ __global__ void __launch_bounds__(GROUPS == 2 ? 320 : (NTW == 1 ? 288 : 160))
     for (int kk = sg.k0; kk < kend; kk += G::STAGE_CHUNKS, ++s) {
       const int slot = s % G::NSTAGES;
       const uint32_t par = (uint32_t)(s / G::NSTAGES) & 1u;
+      if (prefetch_next && kk + G::STAGE_CHUNKS >= kend) {
+#pragma unroll
+        for (int r = 0; r < RPW; ++r) {
+          const uint4* qp = q_ptr(nx_b, nx_hk, r);
+          if (qp) prefetch_l1(qp);
+        }
+      }
       if (!failed && !mbar_wait(&full[slot], par, a.status)) failed = true;
       const int t0 = kk * kChunk;
       const int nvalid = min(min(G::STAGE_CHUNKS, kend - kk) * kChunk, Nb - t0);

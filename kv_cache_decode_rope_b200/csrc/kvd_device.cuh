@@ -119,6 +119,11 @@ __device__ __forceinline__ void cp_async_wait_all() {
 }
 
 // Named barrier over the first `nthreads` threads of the block (id != 0).
+// Bring the cache line holding p into L1 (no register, no wait).
+__device__ __forceinline__ void prefetch_l1(const void* p) {
+  asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
+}
+
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
