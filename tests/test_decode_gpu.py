@@ -264,3 +264,19 @@ def test_repeated_calls_are_deterministic():
     b = gpu_decode(inp, d)
     torch.cuda.synchronize()
     assert torch.equal(a, b)
+
+
+# The CUDA-core kernel runs two CTAs of the split per block for up to 4 rows
+# per unit, while both groups' shared memory and the per-sequence tables fit;
+# a batch this large takes the one-group-per-block launch, a small one leaves
+# the second group of the last block without a CTA (odd grid).
+@pytest.mark.parametrize("batch,len_range", [(1800, (1, 40)), (3, (1, 40))])
+def test_block_group_layouts_match_oracle(batch, len_range):
+    w = WORKLOADS["paged_cb"].with_(batch=batch, num_heads=8, num_kv_heads=2, len_range=len_range,
+                                    paged=False)
+    inp = make_inputs(w, seed=5, fill="nan")
+    _, out = gpu_step(inp, out_dtype=torch.float32)
+    _, _, _, ref = oracle_step(inp)
+    err = oracle.max_abs_diff(np64(out), ref)
+    log_error(f"f32_out[groups_b{batch}]", err)
+    assert err <= tol_for(w), f"max abs diff {err:.3e}"
