@@ -257,9 +257,13 @@ __global__ void __launch_bounds__(GROUPS == 2 ? 320 : (NTW == 1 ? 288 : 160))
   int* sPrefix = reinterpret_cast<int*>(smem_all + S::prefix_off(ncw, GROUPS));
 
   // ---- prologue: clear stages, barriers, per-sequence chunk prefix --------
+  // the lengths' first round trip overlaps the clearing
+  if ((int)threadIdx.x < a.B) prefetch_l1(a.shard_lens ? a.shard_lens + threadIdx.x : a.seq_lens + threadIdx.x);
   {
-    uint4* z = reinterpret_cast<uint4*>(smem);
-    const int n16 = (int)(S::stages() / 16);
+    // V rows past a partial stage meet zero weights, so they must be finite:
+    // the V ring starts from zeros.  K rows there only feed masked scores.
+    uint4* z = reinterpret_cast<uint4*>(sV);
+    const int n16 = (int)(S::stages() / 32);
     for (int k = tid; k < n16; k += gthreads) z[k] = make_uint4(0, 0, 0, 0);
   }
   if (tid == 0) {

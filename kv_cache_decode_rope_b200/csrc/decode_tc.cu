@@ -194,9 +194,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  {  // stale ring contents must be finite: start from zeros
-    uint4* z = reinterpret_cast<uint4*>(sK);
-    for (int k = threadIdx.x; k < (NK + NV) * C::KVSTAGE / 16; k += blockDim.x)
+  // the lengths' first round trip overlaps the clearing
+  if ((int)threadIdx.x < a.B) prefetch_l1(a.shard_lens ? a.shard_lens + threadIdx.x : a.seq_lens + threadIdx.x);
+  {  // V rows past a partial stage meet zero weights, so they must be finite:
+     // the V ring starts from zeros.  K rows there only feed masked scores (and
+     // padding rows, whose output is never written).
+    uint4* z = reinterpret_cast<uint4*>(sV);
+    for (int k = threadIdx.x; k < NV * C::KVSTAGE / 16; k += blockDim.x)
       z[k] = make_uint4(0, 0, 0, 0);
   }
   if (threadIdx.x == 0) {
