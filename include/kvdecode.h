@@ -27,11 +27,12 @@
  * - Stream order with programmatic dependent launch: every kernel of the
  *   library may begin while the kernel before it on the stream finishes,
  *   when that kernel allows early launch (the library's own kernels do).
- *   Before waiting for it, a kernel reads only seq_lens and block_table;
- *   q, k_new, v_new, the caches, out, the workspace and the status word are
- *   touched only after that kernel has completed.  So a preceding kernel
- *   that allows early launch must not write seq_lens or block_table; any
- *   other preceding work is fully ordered as usual.
+ *   Before waiting for it, a kernel reads only seq_lens, block_table and
+ *   (sequence-sharded calls) shard_start / shard_lens, and may OR a flag
+ *   into the status word; q, k_new, v_new, the caches, out and the
+ *   workspace are touched only after that kernel has completed.  So a
+ *   preceding kernel that allows early launch must not write those index
+ *   arrays; any other preceding work is fully ordered as usual.
  *
  * Notation: B = batch, T = q_len (new tokens per sequence), Hq / Hkv = query /
  * key-value heads, g = Hq / Hkv, D = head_dim, L_b = seq_lens[b] = tokens
