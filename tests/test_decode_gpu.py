@@ -270,13 +270,14 @@ def test_repeated_calls_are_deterministic():
 # per unit, while both groups' shared memory and the per-sequence tables fit;
 # a batch this large takes the one-group-per-block launch, a small one leaves
 # the second group of the last block without a CTA (odd grid).
-@pytest.mark.parametrize("batch,len_range", [(1800, (1, 40)), (3, (1, 40))])
-def test_block_group_layouts_match_oracle(batch, len_range):
+@pytest.mark.parametrize("batch,len_range,paged", [(1800, (1, 40), False), (3, (1, 40), False),
+                                                    (24, (1, 3000), True), (900, (1, 40), True)])
+def test_block_group_layouts_match_oracle(batch, len_range, paged):
     w = WORKLOADS["paged_cb"].with_(batch=batch, num_heads=8, num_kv_heads=2, len_range=len_range,
-                                    paged=False)
+                                    paged=paged)
     inp = make_inputs(w, seed=5, fill="nan")
     _, out = gpu_step(inp, out_dtype=torch.float32)
     _, _, _, ref = oracle_step(inp)
     err = oracle.max_abs_diff(np64(out), ref)
-    log_error(f"f32_out[groups_b{batch}]", err)
+    log_error(f"f32_out[groups_b{batch}_{'paged' if paged else 'contig'}]", err)
     assert err <= tol_for(w), f"max abs diff {err:.3e}"
