@@ -38,7 +38,7 @@ struct Conv<__nv_bfloat16> {
 };
 
 template <typename T, int D>
-__global__ void __launch_bounds__(256) append_rope_kernel(AppendArgs a) {
+__global__ void __launch_bounds__(512) append_rope_kernel(AppendArgs a) {
   constexpr int EPV = 16 / (int)sizeof(T);  // elements per 16-byte vector
   constexpr int HALF = D / 2;
   constexpr int VPR = D / EPV;              // 16-byte vectors per head row
@@ -202,9 +202,11 @@ __global__ void __launch_bounds__(256) append_rope_kernel(AppendArgs a) {
 template <typename T>
 cudaError_t launch_t(const AppendArgs& a, cudaStream_t st) {
   const int grid = a.B * a.T;
+  // one 16-byte item per thread where the heads allow (up to 512 threads), so
+  // that every load of the token goes out in the first round trip
   const int work = (a.Hq + a.Hkv) * a.D / 2 + a.Hkv * a.D;  // upper bound on items
   int threads = 32;
-  while (threads < 256 && threads < work / (16 / (int)sizeof(T))) threads *= 2;
+  while (threads < 512 && threads < work / (16 / (int)sizeof(T))) threads *= 2;
   switch (a.D) {
     case 16: return launch_pdl(append_rope_kernel<T, 16>, dim3(grid), dim3(threads), 0, st, a);
     case 32: return launch_pdl(append_rope_kernel<T, 32>, dim3(grid), dim3(threads), 0, st, a);
