@@ -383,7 +383,13 @@ def full_causal_attention(q_raw, k_raw, v_raw, scale: float, base: float,
 
 
 def max_abs_diff(a, b) -> float:
-    """max |a - b| over all elements (generate.rs uses the same measure)."""
+    """max |a_i - b_i| over corresponding elements: the measure of the
+    exactness check in generate.rs ``run``.  The two arrays must have the same
+    shape (no broadcasting: every element is compared with its own
+    counterpart).  A NaN anywhere makes the result NaN, so a comparison
+    ``max_abs_diff(...) <= tol`` fails on it.  Empty arrays differ by 0."""
     a = np.asarray(a, F64)
     b = np.asarray(b, F64)
+    if a.shape != b.shape:
+        raise ValueError(f"max_abs_diff: shapes differ {a.shape} vs {b.shape}")
     return float(np.max(np.abs(a - b))) if a.size else 0.0

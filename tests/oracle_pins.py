@@ -560,4 +560,36 @@ def pin_shard_paged_equals_contiguous(m):
     np.testing.assert_allclose(a[1], b_[1], atol=1e-14)
 
 
+# ------------------------------------------------------------- the comparator
+def pin_max_abs_diff_hand_cases(m):
+    """The exactness measure of generate.rs ``run`` (max |cached - recompute|)
+    on hand-computed cases: the largest difference wins whatever its sign or
+    position, a difference is never averaged, NaN is never skipped (a NaN in a
+    result must fail every ``<= tol`` check), equal arrays differ by exactly 0,
+    empty arrays by 0, and arrays of different shapes are refused rather than
+    broadcast."""
+    assert m.max_abs_diff([1.0, -3.0], [0.0, 0.0]) == 3.0
+    assert m.max_abs_diff([0.0], [-2.0]) == 2.0
+    assert m.max_abs_diff([-5.0, 1.0], [0.0, 0.0]) == 5.0       # a negative difference dominates
+    assert m.max_abs_diff([[0.0, 0.0], [0.0, 7.5]], np.zeros((2, 2))) == 7.5
+    # one large difference among many small ones: max, not mean or sum
+    a = np.zeros(1000)
+    a[637] = 0.25
+    assert m.max_abs_diff(a, np.zeros(1000)) == 0.25
+    b = np.full(1000, 1e-3)
+    assert m.max_abs_diff(b, np.zeros(1000)) == 1e-3
+    x = np.linspace(-4.0, 4.0, 33)
+    assert m.max_abs_diff(x, x) == 0.0
+    assert m.max_abs_diff(np.zeros(0), np.zeros(0)) == 0.0
+    assert math.isnan(m.max_abs_diff([0.0, float("nan")], [0.0, 0.0]))
+    assert math.isnan(m.max_abs_diff([1.0], [float("nan")]))
+    assert not (m.max_abs_diff([float("nan"), 0.0], [0.0, 0.0]) <= 2e-3)
+    try:
+        m.max_abs_diff(np.zeros((4, 1)), np.zeros(4))
+    except ValueError:
+        pass
+    else:
+        raise AssertionError("max_abs_diff broadcast arrays of different shapes")
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

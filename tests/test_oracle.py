@@ -103,6 +103,39 @@ def _append_cow_skipped(*args, **kw):
     return _orig_append(*args, **kw)
 
 
+def _max_diff_signed(a, b):
+    """max (a - b) instead of max |a - b|."""
+    a, b = np.asarray(a, np.float64), np.asarray(b, np.float64)
+    return float(np.max(a - b)) if a.size else 0.0
+
+
+def _max_diff_mean(a, b):
+    """mean |a - b| instead of the max."""
+    a, b = np.asarray(a, np.float64), np.asarray(b, np.float64)
+    return float(np.mean(np.abs(a - b))) if a.size else 0.0
+
+
+def _max_diff_skips_nan(a, b):
+    """NaN-skipping max: a poisoned element would pass every check."""
+    a, b = np.asarray(a, np.float64), np.asarray(b, np.float64)
+    d = np.abs(a - b)
+    return float(np.nanmax(d)) if a.size and not np.isnan(d).all() else 0.0
+
+
+def _max_diff_broadcasts(a, b):
+    """No shape check: mismatched arrays are broadcast against each other."""
+    a, b = np.asarray(a, np.float64), np.asarray(b, np.float64)
+    return float(np.max(np.abs(a - b))) if a.size else 0.0
+
+
+def _max_diff_first_row(a, b):
+    """Compares only the first element along the leading axis."""
+    a, b = np.asarray(a, np.float64), np.asarray(b, np.float64)
+    if a.shape != b.shape:
+        raise ValueError("shapes differ")
+    return float(np.max(np.abs(a[:1] - b[:1]))) if a.size else 0.0
+
+
 _orig_append = kv.append_rope
 _orig_attend = kv.attend
 _orig_attend_partial = kv.attend_partial
@@ -126,6 +159,11 @@ MUTANTS = {
     "partial_lse_natural_log": ("attend_partial", _attend_partial_natural_log),
     "shard_mask_ignores_offset": ("decode_attention_shard", _shard_no_offset),
     "copy_on_write_skipped": ("append_rope", _append_cow_skipped),
+    "max_abs_diff_signed": ("max_abs_diff", _max_diff_signed),
+    "max_abs_diff_mean": ("max_abs_diff", _max_diff_mean),
+    "max_abs_diff_skips_nan": ("max_abs_diff", _max_diff_skips_nan),
+    "max_abs_diff_broadcasts": ("max_abs_diff", _max_diff_broadcasts),
+    "max_abs_diff_first_row": ("max_abs_diff", _max_diff_first_row),
 }
 
 
