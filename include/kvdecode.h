@@ -316,14 +316,17 @@ KVD_API int kvd_merge_partials(const kvd_params* p, const float* part_o, const f
  * the process exits.  The call allocates nothing.
  * - The first call on a device looks up the array's device address and the
  *   SM count (once per device, with that device current); make that first
- *   call before any stream capture.
+ *   call before any stream capture.  The address belongs to the context that
+ *   was current at the lookup: a call made with another context current
+ *   (after cudaDeviceReset, or under a driver-API context) looks it up again
+ *   for that context, so such a call, too, should come before any capture.
  * - All calls on a device share the one array and it keeps the last call's
  *   contents; no part of it needs clearing (every word a call reads is
  *   written earlier in the same call).  Calls that overlap on the GPU (other
  *   streams, other host threads) race on it: serialise them.
  * - Returns KVD_ERR_WORKSPACE when the problem needs more scratch than the
  *   array holds (about (2 * SMs + B * Hkv) * g * q_len * (head_dim + 1) * 4
- *   bytes); other errors as for decode_attention.
+ *   bytes); every other check, and its order, is that of decode_attention.
  */
 #define KVD_STATIC_WORKSPACE_BYTES (16u << 20)
 KVD_API int decode_attention_static(const kvd_params* p, const void* q, const void* k_cache,

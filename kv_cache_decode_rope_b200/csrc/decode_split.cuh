@@ -812,11 +812,11 @@ inline int d_index(int D) {
   return D == 16 ? 0 : D == 32 ? 1 : D == 64 ? 2 : D == 128 ? 3 : D == 256 ? 4 : -1;
 }
 
-// Per (D, row config): devices on which the shared-memory opt-in was set.
+// Per (D, row config): the contexts in which the shared-memory opt-in was set.
 template <typename T, bool PAGED>
-std::atomic<unsigned long long>& smem_attr_flag(int di, int cfg) {
-  static std::atomic<unsigned long long> flags[5][12];
-  return flags[di][cfg];
+PerContextOnce& smem_attr_once(int di, int cfg) {
+  static PerContextOnce once[5][12];
+  return once[di][cfg];
 }
 
 // One launch of the split kernel with `groups` CTAs of the split per block
@@ -829,16 +829,9 @@ cudaError_t launch_groups(const DecodeArgs& a, int nrg, int cfg_idx, cudaStream_
   const size_t smem = S::total(ncw, a.B, GROUPS);
   if (smem > 227 * 1024) return cudaErrorNotSupported;
   auto kern = decode_kernel<T, D, RPW, NTW, PAGED, GROUPS>;
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  cudaError_t e = smem_opt_in(reinterpret_cast<const void*>(kern), 227 * 1024,
+                              smem_attr_once<T, PAGED>(d_index(D), cfg_idx + (GROUPS == 2 ? 6 : 0)));
   if (e != cudaSuccess) return e;
-  auto& flag = smem_attr_flag<T, PAGED>(d_index(D), cfg_idx + (GROUPS == 2 ? 6 : 0));
-  const unsigned long long bit = 1ull << (dev & 63);
-  if (!(flag.load() & bit)) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
-    if (e != cudaSuccess) return e;
-    flag.fetch_or(bit);
-  }
   e = launch_pdl(kern, dim3((a.grid + GROUPS - 1) / GROUPS), dim3(GROUPS * (ncw + 1) * 32), smem,
                  st, a, nrg);
   if (e != cudaSuccess) return e;

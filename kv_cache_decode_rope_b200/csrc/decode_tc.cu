@@ -717,17 +717,10 @@ cudaError_t launch_tc(const DecodeArgs& a, cudaStream_t st) {
   if (!make_map(&mk, a.k_cache, rows) || !make_map(&mv, a.v_cache, rows)) return cudaErrorNotSupported;
   const size_t smem = TcCfg<M>::bytes(a.B);
   if (smem > 227 * 1024) return cudaErrorNotSupported;
-  static std::atomic<unsigned long long> attr_done{0};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  static PerContextOnce attr_once;
+  cudaError_t e = smem_opt_in(reinterpret_cast<const void*>(decode_tc_kernel<PAGED, M>), 227 * 1024,
+                              attr_once);
   if (e != cudaSuccess) return e;
-  const unsigned long long bit = 1ull << (dev & 63);
-  if (!(attr_done.load() & bit)) {
-    e = cudaFuncSetAttribute(decode_tc_kernel<PAGED, M>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             227 * 1024);
-    if (e != cudaSuccess) return e;
-    attr_done.fetch_or(bit);
-  }
   e = launch_pdl(decode_tc_kernel<PAGED, M>, dim3(a.grid), dim3(TC_THREADS), smem, st, a, mk, mv);
   if (e != cudaSuccess) return e;
   const long long warps = (long long)a.B * a.Hkv * a.R;

@@ -1,10 +1,13 @@
 // C-ABI entry points (include/kvdecode.h): argument checks, workspace
 // carve-up, grid sizing, launches.  No allocation, no synchronisation.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <atomic>
 #include <cmath>
 #include <cstdint>
+#include <mutex>
 
 #include "../../include/kvdecode.h"
 #include "kvd_internal.h"
@@ -46,46 +49,14 @@ int check_cache(const kvd_params* p, bool paged) {
 
 std::atomic<int> g_num_sms[64];
 
-int num_sms_current(int* dev_out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
-  *dev_out = dev;
-  if (dev >= 0 && dev < 64) {
-    const int cached = g_num_sms[dev].load();
-    if (cached > 0) return cached;
-  }
-  int n = 0;
-  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
-  if (dev >= 0 && dev < 64) g_num_sms[dev].store(n);
-  return n;
-}
-
-// Checks and argument set-up of a decode call; *nothing = true when there is
-// no work (empty batch or no new tokens).  No CUDA call except device queries.
+// Checks and argument set-up of a decode call with a caller workspace;
+// *nothing = true when there is no work (empty batch or no new tokens).  No
+// CUDA call except device queries.
 int prepare_decode(const kvd_params* p, const void* q, const void* k_cache, const void* v_cache,
                    const int32_t* seq_lens, const int32_t* block_table, void* out,
                    void* workspace, size_t workspace_bytes, DecodeArgs* args, bool* nothing) {
-  *nothing = false;
-  int rc = check_common(p);
-  if (rc != KVD_OK) return rc;
-  const bool paged = block_table != nullptr;
-  rc = check_cache(p, paged);
-  if (rc != KVD_OK) return rc;
-  if (p->out_dtype != KVD_F32 && p->out_dtype != KVD_BF16) return KVD_ERR_INVALID_ARG;
-  if (!std::isfinite(p->scale)) return KVD_ERR_INVALID_ARG;
-  if (p->batch == 0 || p->q_len == 0) {  // nothing to attend
-    *nothing = true;
-    return KVD_OK;
-  }
-  if (p->max_kv_len < 1) return KVD_ERR_INVALID_ARG;
-  if (p->batch > kMaxBatch) return KVD_ERR_UNSUPPORTED;
-  const int g = p->num_heads / p->num_kv_heads;
-  const long long R = (long long)g * p->q_len;
-  if (!decode_supported(p->head_dim, p->dtype == KVD_BF16, (int)(R > kMaxRows ? kMaxRows + 1 : R)))
-    return KVD_ERR_UNSUPPORTED;
-  if (!q || !k_cache || !v_cache || !seq_lens || !out) return KVD_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
-    return KVD_ERR_INVALID_ARG;
+  const int rc = check_decode(p, q, k_cache, v_cache, seq_lens, block_table, out, nothing);
+  if (rc != KVD_OK || *nothing) return rc;
   const size_t need = kvd_workspace_size(p);
   if (!workspace || workspace_bytes < need || !aligned16(workspace)) return KVD_ERR_WORKSPACE;
 
@@ -93,36 +64,11 @@ int prepare_decode(const kvd_params* p, const void* q, const void* k_cache, cons
   const int sms = num_sms_current(&dev);
   if (sms <= 0) return KVD_ERR_CUDA;
 
-  const WorkspaceLayout wl = workspace_layout(p->batch, p->num_kv_heads, (int)R, p->head_dim);
+  DecodeArgs a = decode_args(p, q, k_cache, v_cache, seq_lens, block_table, out, sms);
+  const WorkspaceLayout wl = workspace_layout(p->batch, p->num_kv_heads, a.R, p->head_dim);
   unsigned char* ws = static_cast<unsigned char*>(workspace);
-  DecodeArgs a{};
-  a.q = q;
-  a.k_cache = k_cache;
-  a.v_cache = v_cache;
-  a.seq_lens = seq_lens;
-  a.block_table = block_table;
-  a.out = out;
   a.part_o = reinterpret_cast<float*>(ws + wl.part_o_off);
   a.part_lse = reinterpret_cast<float*>(ws + wl.part_lse_off);
-  a.status = p->status;
-  a.B = p->batch;
-  a.T = p->q_len;
-  a.Hq = p->num_heads;
-  a.Hkv = p->num_kv_heads;
-  a.g = g;
-  a.R = (int)R;
-  a.D = p->head_dim;
-  a.max_seq_len = p->max_seq_len;
-  a.page_size = p->page_size;
-  a.num_pages = p->num_pages;
-  a.max_pages_per_seq = p->max_pages_per_seq;
-  const long long cap =
-      paged ? (long long)p->max_pages_per_seq * p->page_size : (long long)p->max_seq_len;
-  a.cap_tokens = (int)(cap > INT32_MAX ? INT32_MAX : cap);
-  a.qscale = p->scale * 1.4426950408889634f;  // log2(e): softmax evaluated with exp2
-  a.out_bf16 = p->out_dtype == KVD_BF16;
-  a.grid = decode_grid(p->batch, p->num_kv_heads, p->max_kv_len, sms, p->head_dim,
-                             p->dtype == KVD_BF16, (int)R);
   *args = a;
   return KVD_OK;
 }
@@ -205,6 +151,118 @@ int run_append(const kvd_params* p, const AppendArgs& a, void* stream) {
 }
 
 }  // namespace
+
+int num_sms_current(int* dev_out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  *dev_out = dev;
+  if (dev >= 0 && dev < 64) {
+    const int cached = g_num_sms[dev].load();
+    if (cached > 0) return cached;
+  }
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+  if (dev >= 0 && dev < 64) g_num_sms[dev].store(n);
+  return n;
+}
+
+int check_decode(const kvd_params* p, const void* q, const void* k_cache, const void* v_cache,
+                 const int32_t* seq_lens, const int32_t* block_table, const void* out,
+                 bool* nothing) {
+  *nothing = false;
+  int rc = check_common(p);
+  if (rc != KVD_OK) return rc;
+  const bool paged = block_table != nullptr;
+  rc = check_cache(p, paged);
+  if (rc != KVD_OK) return rc;
+  if (p->out_dtype != KVD_F32 && p->out_dtype != KVD_BF16) return KVD_ERR_INVALID_ARG;
+  if (!std::isfinite(p->scale)) return KVD_ERR_INVALID_ARG;
+  if (p->batch == 0 || p->q_len == 0) {  // nothing to attend
+    *nothing = true;
+    return KVD_OK;
+  }
+  if (p->max_kv_len < 1) return KVD_ERR_INVALID_ARG;
+  if (p->batch > kMaxBatch) return KVD_ERR_UNSUPPORTED;
+  const int g = p->num_heads / p->num_kv_heads;
+  const long long R = (long long)g * p->q_len;
+  if (!decode_supported(p->head_dim, p->dtype == KVD_BF16, (int)(R > kMaxRows ? kMaxRows + 1 : R)))
+    return KVD_ERR_UNSUPPORTED;
+  if (!q || !k_cache || !v_cache || !seq_lens || !out) return KVD_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
+    return KVD_ERR_INVALID_ARG;
+  return KVD_OK;
+}
+
+DecodeArgs decode_args(const kvd_params* p, const void* q, const void* k_cache, const void* v_cache,
+                       const int32_t* seq_lens, const int32_t* block_table, void* out, int sms) {
+  const bool paged = block_table != nullptr;
+  const int g = p->num_heads / p->num_kv_heads;
+  const int R = g * p->q_len;
+  DecodeArgs a{};
+  a.q = q;
+  a.k_cache = k_cache;
+  a.v_cache = v_cache;
+  a.seq_lens = seq_lens;
+  a.block_table = block_table;
+  a.out = out;
+  a.status = p->status;
+  a.B = p->batch;
+  a.T = p->q_len;
+  a.Hq = p->num_heads;
+  a.Hkv = p->num_kv_heads;
+  a.g = g;
+  a.R = R;
+  a.D = p->head_dim;
+  a.max_seq_len = p->max_seq_len;
+  a.page_size = p->page_size;
+  a.num_pages = p->num_pages;
+  a.max_pages_per_seq = p->max_pages_per_seq;
+  const long long cap =
+      paged ? (long long)p->max_pages_per_seq * p->page_size : (long long)p->max_seq_len;
+  a.cap_tokens = (int)(cap > INT32_MAX ? INT32_MAX : cap);
+  a.qscale = p->scale * 1.4426950408889634f;  // log2(e): softmax evaluated with exp2
+  a.out_bf16 = p->out_dtype == KVD_BF16;
+  a.grid = decode_grid(p->batch, p->num_kv_heads, p->max_kv_len, sms, p->head_dim,
+                       p->dtype == KVD_BF16, R);
+  return a;
+}
+
+unsigned long long current_context_id() {
+  static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(f);
+    f = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(f);
+  });
+  if (!get_current || !get_id) return 0;
+  CUcontext c = nullptr;
+  if (get_current(&c) != CUDA_SUCCESS || !c) return 0;
+  unsigned long long id = 0;
+  if (get_id(c, &id) != CUDA_SUCCESS) return 0;
+  return id + 1;   // 0 stays "no context"
+}
+
+cudaError_t smem_opt_in(const void* func, int bytes, PerContextOnce& once) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const bool tracked = dev >= 0 && dev < 64;
+  const unsigned long long id = current_context_id();
+  if (tracked && id != 0 && once.ctx[dev].load() == id) return cudaSuccess;
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return e;
+  // the runtime call made a context current if none was
+  if (tracked) once.ctx[dev].store(current_context_id());
+  return cudaSuccess;
+}
 
 WorkspaceLayout workspace_layout(int B, int Hkv, int R, int D) {
   WorkspaceLayout w{};

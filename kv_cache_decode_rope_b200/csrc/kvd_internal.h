@@ -6,6 +6,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "../../include/kvdecode.h"
 
 namespace kvd {
@@ -82,6 +84,34 @@ struct WorkspaceLayout {
   size_t part_lse_off, part_o_off, total;
 };
 WorkspaceLayout workspace_layout(int B, int Hkv, int R, int D);
+
+// Host checks of a decode call, in the order every decode entry point applies
+// them; no CUDA call.  Sets *nothing when there is no work (empty batch or no
+// new tokens), after the checks that do not depend on the work.
+int check_decode(const kvd_params* p, const void* q, const void* k_cache, const void* v_cache,
+                 const int32_t* seq_lens, const int32_t* block_table, const void* out,
+                 bool* nothing);
+// Launch arguments of a checked decode call for `sms` SMs (grid included),
+// except the split partials part_o / part_lse, which the caller points at its
+// scratch.
+DecodeArgs decode_args(const kvd_params* p, const void* q, const void* k_cache, const void* v_cache,
+                       const int32_t* seq_lens, const int32_t* block_table, void* out, int sms);
+// SM count of the current device (cached per device); -1 on a CUDA error.
+int num_sms_current(int* dev_out);
+
+// Unique id of the CUDA context current on the calling thread (never reused
+// by a later context, e.g. after cudaDeviceReset), or 0 when there is none or
+// the driver cannot tell.
+unsigned long long current_context_id();
+
+// One-time set-up of one kernel, per device ordinal: the context id under
+// which it was last done.  A new context (a device reset, a driver-API
+// context) gets the set-up again.
+struct PerContextOnce {
+  std::atomic<unsigned long long> ctx[64] = {};
+};
+// Raise func's dynamic shared-memory limit to `bytes`, once per context.
+cudaError_t smem_opt_in(const void* func, int bytes, PerContextOnce& once);
 
 cudaError_t launch_append(const AppendArgs& a, int bf16, cudaStream_t st);
 // Returns cudaErrorNotSupported when no kernel is compiled for the shape.

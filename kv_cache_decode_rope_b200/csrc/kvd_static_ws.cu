@@ -13,7 +13,6 @@
 // allocating routine.
 #include <cuda_runtime.h>
 
-#include <cmath>
 #include <cstdint>
 #include <mutex>
 
@@ -29,26 +28,33 @@ static __device__ __align__(256) unsigned char g_decode_scratch[KVD_STATIC_WORKS
 
 constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mu;
-void* g_scratch_ptr[kMaxDevices] = {};
-int g_scratch_sms[kMaxDevices] = {};
+// Per device: the context of the last address lookup and the address there.
+// A device address belongs to one context; after a device reset, or with
+// another context current, the array is looked up again.
+struct ScratchAddr {
+  unsigned long long ctx;
+  void* ptr;
+};
+ScratchAddr g_scratch[kMaxDevices] = {};
 
-// Device address of the scratch array and SM count on the current device,
-// looked up once per device (the first call on a device does this set-up).
-int scratch_for_current_device(void** ptr, int* sms) {
+// Device address of the scratch array in the current context.  The first
+// call on a device (or in a new context) asks the runtime for it with that
+// device current; later calls reuse it.
+int scratch_for_current_context(void** ptr) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return KVD_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_ptr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || !p) return KVD_ERR_CUDA;
-    int n = 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
-      return KVD_ERR_CUDA;
-    g_scratch_ptr[dev] = p;
-    g_scratch_sms[dev] = n;
+  const unsigned long long ctx = current_context_id();
+  if (ctx != 0 && g_scratch[dev].ctx == ctx && g_scratch[dev].ptr) {
+    *ptr = g_scratch[dev].ptr;
+    return KVD_OK;
   }
-  *ptr = g_scratch_ptr[dev];
-  *sms = g_scratch_sms[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || !p) return KVD_ERR_CUDA;
+  // the lookup made a context current if none was: record that one
+  g_scratch[dev].ctx = current_context_id();
+  g_scratch[dev].ptr = p;
+  *ptr = p;
   return KVD_OK;
 }
 
@@ -62,75 +68,31 @@ using namespace kvd;
 extern "C" int decode_attention_static(const kvd_params* p, const void* q, const void* k_cache,
                                        const void* v_cache, const int32_t* seq_lens,
                                        const int32_t* block_table, void* out, void* stream) {
-  if (!p) return KVD_ERR_INVALID_ARG;
-  if (p->batch < 0 || p->q_len < 0 || p->num_heads < 1 || p->num_kv_heads < 1 ||
-      p->num_heads % p->num_kv_heads != 0)
-    return KVD_ERR_INVALID_ARG;
-  if (p->dtype != KVD_F32 && p->dtype != KVD_BF16) return KVD_ERR_INVALID_ARG;
-  if (p->out_dtype != KVD_F32 && p->out_dtype != KVD_BF16) return KVD_ERR_INVALID_ARG;
-  if (!std::isfinite(p->scale)) return KVD_ERR_INVALID_ARG;
-  const bool paged = block_table != nullptr;
-  if (paged) {
-    if (p->page_size < kChunk || p->page_size % kChunk != 0) return KVD_ERR_UNSUPPORTED;
-    if (p->num_pages < 1 || p->max_pages_per_seq < 1) return KVD_ERR_INVALID_ARG;
-  } else if (p->max_seq_len < 1) {
-    return KVD_ERR_INVALID_ARG;
-  }
-  if (p->batch == 0 || p->q_len == 0) return KVD_OK;
-  if (p->max_kv_len < 1) return KVD_ERR_INVALID_ARG;
-  if (p->batch > kMaxBatch) return KVD_ERR_UNSUPPORTED;
-  const int g = p->num_heads / p->num_kv_heads;
-  const long long R = (long long)g * p->q_len;
-  if (R > kMaxRows || !decode_supported(p->head_dim, p->dtype == KVD_BF16, (int)R))
-    return KVD_ERR_UNSUPPORTED;
-  if (!q || !k_cache || !v_cache || !seq_lens || !out) return KVD_ERR_INVALID_ARG;
-  const auto mis = [](const void* x) { return (reinterpret_cast<uintptr_t>(x) & 15u) != 0; };
-  if (mis(q) || mis(k_cache) || mis(v_cache) || mis(out)) return KVD_ERR_INVALID_ARG;
+  // the same checks, in the same order, as decode_attention / _paged
+  bool nothing = false;
+  int rc = check_decode(p, q, k_cache, v_cache, seq_lens, block_table, out, &nothing);
+  if (rc != KVD_OK || nothing) return rc;
 
   void* scratch = nullptr;
-  int sms = 0;
-  const int rc = scratch_for_current_device(&scratch, &sms);
+  rc = scratch_for_current_context(&scratch);
   if (rc != KVD_OK) return rc;
+  int dev = 0;
+  const int sms = num_sms_current(&dev);
+  if (sms <= 0) return KVD_ERR_CUDA;
 
   // Carve the scratch for the grid this call launches: one partial slot per
   // (CTA, unit) pair the work split can produce, i.e. grid + units slots.
-  const int grid = decode_grid(p->batch, p->num_kv_heads, p->max_kv_len, sms, p->head_dim,
-                             p->dtype == KVD_BF16, (int)R);
+  DecodeArgs a = decode_args(p, q, k_cache, v_cache, seq_lens, block_table, out, sms);
   const size_t U = (size_t)p->batch * p->num_kv_heads;
-  const size_t slots = (size_t)grid + U;
+  const size_t slots = (size_t)a.grid + U;
   const size_t lse_off = 0;
-  const size_t o_off = align256(lse_off + slots * (size_t)R * sizeof(float));
-  const size_t need = align256(o_off + slots * (size_t)R * p->head_dim * sizeof(float));
+  const size_t o_off = align256(lse_off + slots * (size_t)a.R * sizeof(float));
+  const size_t need = align256(o_off + slots * (size_t)a.R * a.D * sizeof(float));
   if (need > (size_t)KVD_STATIC_WORKSPACE_BYTES) return KVD_ERR_WORKSPACE;
 
   unsigned char* ws = static_cast<unsigned char*>(scratch);
-  DecodeArgs a{};
-  a.q = q;
-  a.k_cache = k_cache;
-  a.v_cache = v_cache;
-  a.seq_lens = seq_lens;
-  a.block_table = block_table;
-  a.out = out;
   a.part_o = reinterpret_cast<float*>(ws + o_off);
   a.part_lse = reinterpret_cast<float*>(ws + lse_off);
-  a.status = p->status;
-  a.B = p->batch;
-  a.T = p->q_len;
-  a.Hq = p->num_heads;
-  a.Hkv = p->num_kv_heads;
-  a.g = g;
-  a.R = (int)R;
-  a.D = p->head_dim;
-  a.max_seq_len = p->max_seq_len;
-  a.page_size = p->page_size;
-  a.num_pages = p->num_pages;
-  a.max_pages_per_seq = p->max_pages_per_seq;
-  const long long cap =
-      paged ? (long long)p->max_pages_per_seq * p->page_size : (long long)p->max_seq_len;
-  a.cap_tokens = (int)(cap > INT32_MAX ? INT32_MAX : cap);
-  a.qscale = p->scale * 1.4426950408889634f;
-  a.out_bf16 = p->out_dtype == KVD_BF16;
-  a.grid = grid;
   const cudaError_t e = launch_decode(a, p->dtype == KVD_BF16, static_cast<cudaStream_t>(stream));
   if (e == cudaErrorNotSupported) return KVD_ERR_UNSUPPORTED;
   return e == cudaSuccess ? KVD_OK : KVD_ERR_CUDA;

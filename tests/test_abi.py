@@ -153,3 +153,43 @@ def test_workspace_size_grows_with_problem(lib):
     rows = lib.kvd_workspace_size(ctypes.byref(params(q_len=4)))
     assert 0 < small < big
     assert rows > lib.kvd_workspace_size(ctypes.byref(params()))
+
+
+def call_static(lib, p, q=FAKE, paged=False):
+    return lib.decode_attention_static(ctypes.byref(p), q, FAKE, FAKE, FAKE, FAKE if paged else None,
+                                       FAKE, None)
+
+
+STATIC_CASES = [
+    dict(num_heads=6, num_kv_heads=4), dict(num_kv_heads=0), dict(head_dim=96),
+    dict(head_dim=256, dtype=_lib.KVD_F32), dict(dtype=7), dict(out_dtype=3),
+    dict(num_heads=256, num_kv_heads=1), dict(num_heads=128, num_kv_heads=1, dtype=_lib.KVD_F32),
+    dict(max_seq_len=0), dict(max_kv_len=0), dict(scale=float("nan")),
+    # no work, but a configuration no kernel supports: refused all the same
+    dict(batch=0, head_dim=48), dict(q_len=0, head_dim=96), dict(batch=0, dtype=7),
+    dict(batch=0, max_seq_len=0),
+]
+
+
+@pytest.mark.parametrize("kw", STATIC_CASES)
+def test_static_entry_validates_like_decode_attention(lib, kw):
+    """decode_attention_static answers every rejected configuration exactly as
+    decode_attention does, before any CUDA call (these run without a GPU)."""
+    p = params(**kw)
+    ref = lib.decode_attention(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 30, None)
+    assert ref != 0
+    assert call_static(lib, p) == ref
+
+
+@pytest.mark.parametrize("kw", [dict(page_size=8), dict(num_pages=0), dict(max_pages_per_seq=0)])
+def test_static_entry_paged_validation(lib, kw):
+    p = params(**kw)
+    assert call_static(lib, p, paged=True) == call_decode(lib, p, paged=True) != 0
+
+
+def test_static_entry_pointer_checks_and_empty_calls(lib):
+    assert lib.decode_attention_static(None, FAKE, FAKE, FAKE, FAKE, None, FAKE, None) == -1
+    assert call_static(lib, params(), q=0) == -1
+    assert call_static(lib, params(), q=FAKE + 2) == -1
+    assert call_static(lib, params(batch=0)) == 0
+    assert call_static(lib, params(q_len=0), paged=True) == 0

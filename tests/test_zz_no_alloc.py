@@ -4,9 +4,11 @@ latency-critical path where an allocation would synchronise the device, a
 foreign-function caller without a device allocator).  It keeps its split
 scratch in an array inside the library instead of a caller workspace.
 
-Checked through the C ABI against the workspace entry points, on two calls in
-a row with different inputs (the shared array keeps the first call's
-contents, which must not leak into the second).  This file is collected last
+Checked through the C ABI against the workspace entry points, bit for bit, on
+two calls in a row with different inputs (the shared array keeps the first
+call's contents, which must not leak into the second), against the fp64 oracle,
+and for not allocating: the second call leaves the device's free memory as it
+was.  This file is collected last
 so that a stop at the first failure has already run every other test."""
 import ctypes
 
@@ -14,12 +16,13 @@ import pytest
 import torch
 
 import kv_cache_decode_rope_b200 as kvd
+import oracle
 from kv_cache_decode_rope_b200 import _lib
 from kv_cache_decode_rope_b200.workloads import WORKLOADS, make_inputs
 
 pytestmark = pytest.mark.gpu
 
-TOL = 2e-3   # the bf16-input tolerance the parity tests use
+TOL = 2e-3   # the bf16-input tolerance the parity tests use (fp32 output vs the fp64 oracle)
 
 CASES = {
     "contiguous": WORKLOADS["batched_gqa"].with_(batch=4, cache_len=3000),
@@ -44,6 +47,17 @@ def _params(w, d, mkl):
                            out_dtype=torch.float32, max_kv_len=mkl, **paging)
 
 
+def oracle_step_no_append(host):
+    """The oracle's decode of the cache as drawn (no append: the static call
+    attends the cache it is given)."""
+    w = host["workload"]
+    f64 = lambda t: t.float().numpy().astype("float64")  # noqa: E731
+    bt = None if host["block_table"] is None else host["block_table"].numpy()
+    q = f64(host["q"])
+    kc, vc = f64(host["k_cache"]), f64(host["v_cache"])
+    return q, kc, vc, oracle.decode_attention(q, kc, vc, host["seq_lens"].numpy(), w.scale, bt)
+
+
 def _call_static(p, d, out):
     lib = _lib.get_lib()
     bt = d["block_table"]
@@ -53,28 +67,51 @@ def _call_static(p, d, out):
                                        torch.cuda.current_stream().cuda_stream)
 
 
+def _workspace_call(w, d, mkl):
+    if d["block_table"] is None:
+        return kvd.decode_attention(d["q"], d["k_cache"], d["v_cache"], d["seq_lens"], scale=w.scale,
+                                    max_kv_len=mkl, out_dtype=torch.float32)
+    return kvd.decode_attention_paged(d["q"], d["k_cache"], d["v_cache"], d["seq_lens"],
+                                      d["block_table"], scale=w.scale, max_kv_len=mkl,
+                                      out_dtype=torch.float32)
+
+
 @pytest.mark.parametrize("name", sorted(CASES))
 def test_static_scratch_matches_workspace_entry_point(name):
+    """Two static calls in a row, on different inputs, each bit for bit equal
+    to the workspace entry point: the same kernels with the same grid and the
+    same arithmetic per partial slot, so any difference would be stale or
+    misplaced scratch.  The second call is also checked against the fp64
+    oracle, and it must leave the device's free memory and torch's
+    allocations unchanged (it allocates nothing)."""
     w = CASES[name]
     runs = []
     for seed in (31, 32):   # two different inputs for the two calls in a row
-        d = _device(make_inputs(w, seed=seed, fill="zero"))
+        host = make_inputs(w, seed=seed, fill="zero")
+        d = _device(host)
         mkl = int(d["seq_lens"].max()) + w.q_len
-        if d["block_table"] is None:
-            ref = kvd.decode_attention(d["q"], d["k_cache"], d["v_cache"], d["seq_lens"], scale=w.scale,
-                                       max_kv_len=mkl, out_dtype=torch.float32)
-        else:
-            ref = kvd.decode_attention_paged(d["q"], d["k_cache"], d["v_cache"], d["seq_lens"],
-                                             d["block_table"], scale=w.scale, max_kv_len=mkl,
-                                             out_dtype=torch.float32)
-        runs.append((d, ref, _params(w, d, mkl), torch.full_like(ref, float("nan"))))
+        ref = _workspace_call(w, d, mkl)
+        runs.append((host, d, ref, _params(w, d, mkl), torch.full_like(ref, float("nan"))))
     torch.cuda.synchronize()
-    for d, _, p, out in runs:            # the two static calls back to back
-        assert _call_static(p, d, out) == _lib.KVD_OK
+    # first static call: resolves the array's address (once per device)
+    _, d0, _, p0, out0 = runs[0]
+    assert _call_static(p0, d0, out0) == _lib.KVD_OK
     torch.cuda.synchronize()
-    for d, ref, _, out in runs:
+    free0, _ = torch.cuda.mem_get_info()
+    alloc0 = torch.cuda.memory_allocated()
+    _, d1, _, p1, out1 = runs[1]
+    assert _call_static(p1, d1, out1) == _lib.KVD_OK
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0, f"a static call changed free device memory by {free0 - free1} bytes"
+    assert torch.cuda.memory_allocated() == alloc0
+    for _, _, ref, _, out in runs:
         assert torch.isfinite(out).all()
-        assert (out - ref).abs().max().item() <= TOL
+        assert torch.equal(out, ref)
+    host, _, _, _, out = runs[1]
+    _, _, _, ref64 = oracle_step_no_append(host)
+    err = oracle.max_abs_diff(out.cpu().double().numpy(), ref64)
+    assert err <= TOL, f"{name}: max abs diff vs the oracle {err:.3e}"
 
 
 def test_static_scratch_rejects_oversized_problems():
