@@ -8,7 +8,12 @@ workload, so no flush is needed between steps (the tiny workload is flushed).
 ``value`` is algorithmic bytes per step (see workloads.step_bytes) divided by
 the device time of the step, summed over ranks; ``e2e`` times the same step
 through the public API with the new tokens copied from pinned host memory and
-the output copied back, inside the timed region.
+the output copied back, inside the timed region.  ``roofline`` is the decode
+call alone (split-KV kernel + merge), with the mean, median and p10/p90 of its
+per-launch device times.  ``workloads`` repeats the device timings (decode
+median/p10/p90, step, algorithmic bytes, fraction of the measured copy peak,
+clocks) for every other workload in the same run.  ``cpu_baseline`` is the
+fp64 oracle on the host cores, on all BLAS threads and on one.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
                     [--impl ours|reference]
@@ -39,13 +44,15 @@ L2_BYTES = 126 * 1024 * 1024
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="batched_gqa")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="CPU time budget of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="time only --workload (default: every other workload too, in a 'workloads' object)")
     ap.add_argument("--cascade", action="store_true",
                     help="shared_prefix workload: decode as prefix-once-per-group + suffix + merge "
                          "(kv_cache_decode_rope_b200.prefix.cascade_decode)")
@@ -167,19 +174,24 @@ class ClockSampler:
 _UNIT_POOL = {}
 
 
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:  # noqa: BLE001
+        return 1
+
+
 def oracle_sample(w, seconds: float, seed: int):
     """Time the fp64 oracle's decode on host cores over a bounded sample of the
     workload: whole (sequence, kv head) units, one after another, until the
-    time budget is spent.  Returns (GB/s of attended K/V bytes, cores, text)."""
+    time budget is spent.  Returns (GB/s of attended K/V bytes, threads used,
+    text)."""
     import numpy as np
     import torch
     import oracle
     from kv_cache_decode_rope_b200.workloads import draw_lengths
-    try:
-        from threadpoolctl import threadpool_info
-        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-    except Exception:  # noqa: BLE001
-        cores = 1
+    cores = blas_threads()
     gen = torch.Generator().manual_seed(seed)
     lens = draw_lengths(w, gen)
     g, D, T = w.group, w.head_dim, w.q_len
@@ -211,15 +223,49 @@ def oracle_sample(w, seconds: float, seed: int):
         f"fp64 oracle attend, {elapsed:.1f} s of CPU time")
 
 
+def cpu_baseline(w, seconds: float, seed: int) -> dict:
+    """The oracle on the host cores: all BLAS threads, then one thread."""
+    v, cores, sample = oracle_sample(w, seconds, seed)
+    res = {"value": round(v, 4), "unit": "GB/s", "cores": cores, "cores_total": os.cpu_count(),
+           "kind": "oracle", "sample": sample}
+    try:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1):
+            v1, _, sample1 = oracle_sample(w, seconds / 2, seed)
+        res["single_thread"] = {"value": round(v1, 4), "unit": "GB/s", "cores": 1, "sample": sample1}
+    except Exception as e:  # noqa: BLE001 - reported, not fatal
+        res["single_thread"] = {"unavailable": str(e)[:120]}
+    return res
+
+
 # ------------------------------------------------------------------ GPU bench
-def run_ours(args, rank, world, local):
+def pct(xs, q):
+    """q-th percentile (0..100) of xs by linear interpolation."""
+    xs = sorted(xs)
+    if not xs:
+        return None
+    k = (len(xs) - 1) * q / 100.0
+    lo = int(math.floor(k))
+    hi = min(lo + 1, len(xs) - 1)
+    return xs[lo] + (xs[hi] - xs[lo]) * (k - lo)
+
+
+def dist_us(ms):
+    """median, p10, p90 and mean of per-iteration times (ms) in µs."""
+    return {"median": round(1e3 * statistics.median(ms), 2), "p10": round(1e3 * pct(ms, 10), 2),
+            "p90": round(1e3 * pct(ms, 90), 2), "mean": round(1e3 * sum(ms) / len(ms), 2),
+            "n": len(ms)}
+
+
+def measure(args, w, local, rank, world, steps, kernel_iters, e2e=False, cascade=False):
+    """All device timings of one workload: K steps (append + decode) as the
+    timed region, then per-call loops of the decode and the append, and, for
+    the headline, the end-to-end step through pinned host memory."""
     import torch
     import kv_cache_decode_rope_b200 as kvd
-    from kv_cache_decode_rope_b200.workloads import WORKLOADS, make_inputs_device, step_bytes
+    from kv_cache_decode_rope_b200.workloads import make_inputs_device, step_bytes
 
-    torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    w = WORKLOADS[args.workload]
     if w.cache_mode == "prefill":
         w = w.with_(cache_mode="random")
     inp = make_inputs_device(w, seed=1000 + w.config_id + 7919 * rank, device=dev)
@@ -237,25 +283,25 @@ def run_ours(args, rank, world, local):
     flush = cache_bytes < 2 * L2_BYTES
     flush_buf = torch.empty(4 * L2_BYTES // 4, dtype=torch.int32, device=dev) if flush else None
 
-    def append(q, kn, vn, seq):
-        kvd.append_rope(q, kn, vn, inp["k_cache"], inp["v_cache"], seq, bt, rope_base=w.rope_base,
-                        status=status)
+    def append(q, kn, vn, seq, bt_=bt, st=status):
+        kvd.append_rope(q, kn, vn, inp["k_cache"], inp["v_cache"], seq, bt_, rope_base=w.rope_base,
+                        status=st)
 
-    if args.cascade and not w.shared_prefix:
+    if cascade and not w.shared_prefix:
         raise SystemExit("--cascade needs a workload with a shared prefix")
 
-    def decode(q, seq):
-        if args.cascade:
+    def decode(q, seq, bt_=bt, st=status):
+        if cascade:
             from kv_cache_decode_rope_b200.prefix import cascade_decode
-            cascade_decode(q, inp["k_cache"], inp["v_cache"], seq, bt, w.shared_prefix,
+            cascade_decode(q, inp["k_cache"], inp["v_cache"], seq, bt_, w.shared_prefix,
                            scale=w.scale, out=out)
             return
-        if bt is None:
+        if bt_ is None:
             kvd.decode_attention(q, inp["k_cache"], inp["v_cache"], seq, out, scale=w.scale,
-                                 max_kv_len=mkl, workspace=ws, status=status)
+                                 max_kv_len=mkl, workspace=ws, status=st)
         else:
-            kvd.decode_attention_paged(q, inp["k_cache"], inp["v_cache"], seq, bt, out, scale=w.scale,
-                                       max_kv_len=mkl, workspace=ws, status=status)
+            kvd.decode_attention_paged(q, inp["k_cache"], inp["v_cache"], seq, bt_, out, scale=w.scale,
+                                       max_kv_len=mkl, workspace=ws, status=st)
 
     q, kn, vn, seq = inp["q"], inp["k_new"], inp["v_new"], inp["seq_lens"]
     for _ in range(args.warmup):
@@ -271,6 +317,7 @@ def run_ours(args, rank, world, local):
     # the tail of the one before.  Two more loops replay the decode call and
     # the append call alone to time them separately (the per-kernel figures).
     # --launch eager times plain calls instead.
+    graphs = []
     if args.launch == "graph":
         side = torch.cuda.Stream(device=dev)
         side.wait_stream(torch.cuda.current_stream())
@@ -288,6 +335,7 @@ def run_ours(args, rank, world, local):
         with torch.cuda.graph(g_dec):
             decode(q, seq)
         torch.cuda.synchronize()
+        graphs = [g_step, g_app, g_dec]
         run_step, run_append, run_decode = g_step.replay, g_app.replay, g_dec.replay
         for _ in range(3):
             run_step()
@@ -322,8 +370,13 @@ def run_ours(args, rank, world, local):
         torch.cuda.synchronize()
         return [e0.elapsed_time(e1) for e0, e1 in evs]
 
-    K = args.steps
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    # The timed region: K steps back to back, bracketed by two events (an
+    # event between steps would itself cost the stream several microseconds).
+    # A workload that fits in L2 is flushed before every step instead, and its
+    # steps are then timed one by one, the flush outside each event pair.
+    K = steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K if flush else 0)]
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
@@ -334,21 +387,27 @@ def run_ours(args, rank, world, local):
         for k in range(K):
             if flush:
                 flush_buf.add_(1)
-            ev[k][0].record()
+                ev[k][0].record()
             run_step()
-            ev[k][1].record()
+            if flush:
+                ev[k][1].record()
         t_all1.record()
         torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
-    step_ms = [e0.elapsed_time(e1) for e0, e1 in ev]
-    total_ms = sum(step_ms) if flush else t_all0.elapsed_time(t_all1)
-    # per-kernel figures, outside the timed region
-    Kk = min(K, 200)
-    dec_ms = timed(run_decode, Kk, before=run_append)
-    app_ms = timed(run_append, Kk, before=run_decode)
+        if world > 1:
+            torch.distributed.barrier()
+        total_ms = sum(e0.elapsed_time(e1) for e0, e1 in ev) if flush else t_all0.elapsed_time(t_all1)
+        # per-step and per-kernel figures, after the timed region (clocks still sampled)
+        step_ms = timed(run_step, kernel_iters)
+        dec_ms = timed(run_decode, kernel_iters, before=run_append)
+        app_ms = timed(run_append, kernel_iters, before=run_decode)
     if status.item() != 0:
-        raise RuntimeError(f"device status flags set during the bench: {status.item()}")
+        raise RuntimeError(f"device status flags set during the bench of {w.name}: {status.item()}")
+
+    res = dict(total_ms=total_ms, steps=K, step_ms=step_ms, dec_ms=dec_ms, app_ms=app_ms, bytes=nbytes,
+               clocks=clk.summary(), flush=flush, cache_bytes=cache_bytes, w=w, mkl=mkl)
+    if not e2e:
+        del graphs
+        return res
 
     # ---- end to end: pinned host inputs -> device, step, output -> host
     hq = q.cpu().pin_memory()
@@ -369,41 +428,52 @@ def run_ours(args, rank, world, local):
         ds.copy_(hs, non_blocking=True)
         if dbt is not None:
             dbt.copy_(hbt, non_blocking=True)
-        kvd.append_rope(dq, dk, dv, inp["k_cache"], inp["v_cache"], ds, dbt, rope_base=w.rope_base)
-        if args.cascade:
-            from kv_cache_decode_rope_b200.prefix import cascade_decode
-            cascade_decode(dq, inp["k_cache"], inp["v_cache"], ds, dbt, w.shared_prefix, scale=w.scale,
-                           out=out)
-        elif dbt is None:
-            kvd.decode_attention(dq, inp["k_cache"], inp["v_cache"], ds, out, scale=w.scale,
-                                 max_kv_len=mkl, workspace=ws)
-        else:
-            kvd.decode_attention_paged(dq, inp["k_cache"], inp["v_cache"], ds, dbt, out, scale=w.scale,
-                                       max_kv_len=mkl, workspace=ws)
+        append(dq, dk, dv, ds, dbt, None)
+        decode(dq, ds, dbt, None)
         hout.copy_(out, non_blocking=True)
 
-    for _ in range(max(3, args.warmup // 4)):
+    for _ in range(max(3, args.warmup)):
         e2e_step()
     torch.cuda.synchronize()
-    Ke = max(3, K // 4)
+    Ke = max(K, 20)
     if world > 1:
         torch.distributed.barrier()
+    e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(Ke)]
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record()
-    for _ in range(Ke):
+    for a, b in e_ev:
         if flush:
             flush_buf.add_(1)
+        a.record()
         e2e_step()
+        b.record()
     e1.record()
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / Ke
-
-    res = dict(total_ms=total_ms, step_ms=statistics.median(step_ms),
-               mean_step_ms=total_ms / K, dec_ms=sum(dec_ms) / len(dec_ms), dec_med=statistics.median(dec_ms),
-               app_ms=sum(app_ms) / len(app_ms), e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, bytes=nbytes,
-               clocks=clk.summary(), flush=flush, cache_bytes=cache_bytes, w=w, mkl=mkl)
+    e2e_each = [a.elapsed_time(b) for a, b in e_ev]
+    res.update(e2e_ms=(sum(e2e_each) if flush else e0.elapsed_time(e1)) / Ke, e2e_each=e2e_each,
+               e2e_steps=Ke, h2d=h2d, d2h=d2h)
+    del graphs
     return res
+
+
+def summarise(r, peak) -> dict:
+    """The per-workload figures of one measure() result (device times)."""
+    dec = dist_us(r["dec_ms"])
+    step = dist_us(r["step_ms"])
+    b = r["bytes"]
+    # means: CUDA event times come in steps of about 2 us, so a median of
+    # per-launch times is quantised while a mean over many launches is not
+    gbs = b["decode"] / (dec["mean"] * 1e-6) / 1e9
+    step_region_us = r["total_ms"] * 1e3 / r["steps"]
+    return {"config": workload_config(r["w"], {"max_kv_len": r["mkl"]}),
+            "decode_us": dec, "step_us": step, "append_us": dist_us(r["app_ms"]),
+            "step_us_timed_region": round(step_region_us, 2),
+            "algorithmic_bytes": {"decode": b["decode"], "step": b["step"]},
+            "decode_gbs": round(gbs, 1), "frac": round(gbs / peak, 4),
+            "step_frac": round(b["step"] / (step_region_us * 1e-6) / 1e9 / peak, 4),
+            "l2": "flushed between iterations" if r["flush"] else "inputs larger than L2",
+            "clocks": r["clocks"]}
 
 
 def reduce_max(x: float, world: int) -> float:
@@ -481,17 +551,23 @@ def main():
                                              device_id=torch.device("cuda", local))
     if args.shard_seq:
         return main_sharded(args, rank, world, local)
-    r = run_ours(args, rank, world, local)
-    w = r["w"]
+    from kv_cache_decode_rope_b200.workloads import WORKLOADS
+    torch.cuda.set_device(local)
     K = args.steps
+    kernel_iters = max(K, 200)
+    r = measure(args, WORKLOADS[args.workload], local, rank, world, K, kernel_iters, e2e=True,
+                cascade=args.cascade)
+    w = r["w"]
+    peak, peak_kind = measured_peaks()
     total_ms = reduce_max(r["total_ms"], world)
-    dec_ms = reduce_max(r["dec_ms"], world)
+    dec = dist_us(r["dec_ms"])
+    dec_mean_ms = reduce_max(dec["mean"] * 1e-3, world)
+    dec_med_ms = reduce_max(dec["median"] * 1e-3, world)
     e2e_ms = reduce_max(r["e2e_ms"], world)
     ms_step = total_ms / K
     step_bytes = r["bytes"]["step"]
     value = world * step_bytes / (ms_step * 1e-3) / 1e9
-    peak, peak_kind = measured_peaks()
-    dec_gbs = r["bytes"]["decode"] / (dec_ms * 1e-3) / 1e9
+    dec_gbs = r["bytes"]["decode"] / (dec_mean_ms * 1e-3) / 1e9
     traffic = committed_traffic(w.name)
     line = {
         "metric": METRIC,
@@ -517,6 +593,7 @@ def main():
                                            "decode_attention" + ("_paged" if w.paged else "")),
             "launch": "CUDA graph replay of the two library calls" if args.launch == "graph" else "eager calls",
             "max_kv_len": r["mkl"]}),
+        "step_us": dist_us(r["step_ms"]),
         "roofline": {
             "bound": "hbm",
             "kernel": "decode_attention (split-KV kernel + LSE merge)",
@@ -525,23 +602,47 @@ def main():
             "peak_source": f"{peak_kind} hbm_gbs",
             "unit": "GB/s",
             "frac": round(dec_gbs / peak, 4),
-            "us_per_launch": round(dec_ms * 1e3, 2),
+            "us_per_launch": round(dec_mean_ms * 1e3, 2),
+            "us_per_launch_median": round(dec_med_ms * 1e3, 2),
+            "us_per_launch_p10": dec["p10"],
+            "us_per_launch_p90": dec["p90"],
+            "launches_timed": dec["n"],
+            "frac_median": round(r["bytes"]["decode"] / (dec_med_ms * 1e-3) / 1e9 / peak, 4),
             "algorithmic_bytes_per_launch": r["bytes"]["decode"],
             "traffic": traffic,
         },
-        "append_us": round(r["app_ms"] * 1e3, 2),
+        "append_us": dist_us(r["app_ms"]),
         "e2e": {"value": round(world * step_bytes / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
                 "us_per_step": round(e2e_ms * 1e3, 2),
+                "us_per_step_median": round(1e3 * statistics.median(r["e2e_each"]), 2),
+                "steps": r["e2e_steps"],
                 "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
         "gpu_launches": (6 if args.cascade else 3) * K,
         "clocks": r["clocks"],
     }
+    del r
+    torch.cuda.empty_cache()
+    # Every other workload of the contract, measured in the same run (device
+    # times; per-GPU figures, max over ranks).  Parity-only at the tiny size.
+    if not args.no_workloads and not args.cascade:
+        extra = {}
+        for name in ("batched_gqa", "paged_cb", "mtp_verify", "long_ctx", "tiny_mha"):
+            if name == w.name:
+                continue
+            rw = measure(args, WORKLOADS[name], local, rank, world, K, kernel_iters)
+            sm = summarise(rw, peak)
+            for key in ("decode_us", "step_us"):
+                for stat in ("median", "mean"):
+                    sm[key][stat] = round(1e3 * reduce_max(sm[key][stat] * 1e-3, world), 2)
+            sm["step_us_timed_region"] = round(1e3 * reduce_max(sm["step_us_timed_region"] * 1e-3, world), 2)
+            del rw
+            torch.cuda.empty_cache()
+            extra[name] = sm
+        line["workloads"] = extra
     if args.driver_layers > 0:
         line["driver"] = time_driver(w, args.driver_layers, local)
     if rank == 0 and not args.no_cpu_baseline:
-        v, cores, sample = oracle_sample(w, args.cpu_seconds, seed=1000 + w.config_id)
-        line["cpu_baseline"] = {"value": round(v, 4), "unit": "GB/s", "cores": cores,
-                                "kind": "oracle", "sample": sample}
+        line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds, seed=1000 + w.config_id)
     if world > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
@@ -692,7 +793,8 @@ def main_reference(args, rank, world):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic", "config": workload_config(w),
-        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": info[0], "kind": "oracle",
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": info[0],
+                         "cores_total": os.cpu_count(), "kind": "oracle",
                          "sample": "each step: " + info[1]},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }

@@ -21,7 +21,8 @@
 //   halves h of the stage into two TMEM accumulators, as soon as each half of
 //   P is written; it never waits on the next stage's keys.
 //   P is passed as a bf16 high part (the top 16 bits of the fp32 value) plus
-//   a bf16 residual, which keeps each probability to within 2^-14 relative.
+//   the exact remainder rounded to the nearest bf16, which keeps each
+//   probability to within 2^-15 relative.
 //   With MQ = 64 the two parts are stacked into the 128 rows of one M = 128
 //   product (an M = 64 MMA runs at half the rate of an M = 128 one), and the
 //   epilogue adds the two output rows; with MQ = 128 they are two passes.
@@ -100,6 +101,7 @@ __device__ __forceinline__ void tc_loader(const DecodeArgs& a, const int* sPrefi
   const int lane = threadIdx.x & 31;
   int g = 0;
   bool failed = false;
+  bool waited = false;   // programmatic-dependency wait done (before the first copy)
   // page id of chunk `ch` of sequence b (paged layout), -1 past `kend`
   auto page_of = [&](int b, int ch, int kend) -> int {
     if (ch >= kend) return -1;
@@ -129,6 +131,10 @@ __device__ __forceinline__ void tc_loader(const DecodeArgs& a, const int* sPrefi
       if (lane == 0) ok = mbar_wait(&emptyb[slot], ((uint32_t)(g / NSLOT) & 1u) ^ 1u, a.status);
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) { failed = true; break; }
+      if (!waited) {   // the caches are read only once the previous kernel is done
+        grid_dep_wait();
+        waited = true;
+      }
       const int nck = min(CH, kend - kk);
       int page = -1;
       if (PAGED) page = __shfl_sync(0xffffffffu, win0, kk - wbase + min(lane, CH - 1));
@@ -237,8 +243,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *sTmem;
-  grid_dep_wait();      // q, the caches and the workspace are ready
   grid_dep_launch();
+  // Each role waits for the previous kernel (griddepcontrol.wait) itself, just
+  // before its first access to q, the caches or the outputs: the loaders
+  // before their first copy (their first block-table reads go out before it),
+  // the softmax warps before the q load.  The two MMA issuers touch only
+  // shared and tensor memory and never wait.
 
   const long long total = (long long)a.Hkv * sPrefix[a.B];
   const long long x0 = total * blockIdx.x / a.grid;
@@ -406,6 +416,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(q_full);
       };
+      grid_dep_wait();      // q and the outputs: only after the previous kernel
       issue_q(st.b, st.hk);
       publish_q();
       int Nb_cur = attended_len(a, st.b, false);
@@ -499,7 +510,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             m = mx;
             l *= alpha;
           }
-          uint32_t pk[16], pl[16];   // bf16 pairs: high part (top 16 bits), residual (top 16 bits)
+          uint32_t pk[16], pl[16];   // bf16 pairs: high part (top 16 bits), residual (rounded)
           if (warp_rows) {
             const float mref = (m == -INFINITY) ? 0.f : m;
             const float2 qs2 = make_float2(qs, qs), nm2 = make_float2(-mref, -mref);
@@ -514,7 +525,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
               const float2 hi = make_float2(__uint_as_float(b0 & 0xffff0000u), __uint_as_float(b1 & 0xffff0000u));
               const float2 lo = __ffma2_rn(hi, make_float2(-1.f, -1.f), pp);   // exact: pp - hi
               pk[j] = hi16x2(b0, b1);
-              pl[j] = hi16x2(__float_as_uint(lo.x), __float_as_uint(lo.y));
+              pl[j] = pack_bf16x2(lo.x, lo.y);   // residual rounded to nearest
             }
             l += sum2.x + sum2.y;
           } else {
