@@ -51,6 +51,10 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="CPU time budget of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override the workload's batch (profiling captures of a smaller case)")
+    ap.add_argument("--kernel-iters", type=int, default=0,
+                    help="iterations of the per-kernel loops after the timed region (default max(K, 200))")
     ap.add_argument("--no-workloads", action="store_true",
                     help="time only --workload (default: every other workload too, in a 'workloads' object)")
     ap.add_argument("--cascade", action="store_true",
@@ -554,9 +558,11 @@ def main():
     from kv_cache_decode_rope_b200.workloads import WORKLOADS
     torch.cuda.set_device(local)
     K = args.steps
-    kernel_iters = max(K, 200)
-    r = measure(args, WORKLOADS[args.workload], local, rank, world, K, kernel_iters, e2e=True,
-                cascade=args.cascade)
+    kernel_iters = args.kernel_iters if args.kernel_iters > 0 else max(K, 200)
+    head_w = WORKLOADS[args.workload]
+    if args.batch > 0:
+        head_w = head_w.with_(batch=args.batch)
+    r = measure(args, head_w, local, rank, world, K, kernel_iters, e2e=True, cascade=args.cascade)
     w = r["w"]
     peak, peak_kind = measured_peaks()
     total_ms = reduce_max(r["total_ms"], world)

@@ -13,12 +13,13 @@ from tests.gpu_util import (gpu_append, gpu_decode, gpu_step, log_error, np64, o
                             to_device, tol_for)
 
 # fp32 error allowed on top of one bf16 ulp when comparing a bf16 output: the
-# CUDA-core path accumulates in fp32 (errors ~1e-7); the tensor-core path
-# (g * q_len >= 8, bf16, D = 128) feeds each probability to the MMA as a bf16
-# high part plus a bf16 residual (relative error below 2^-15 per weight) and
-# accumulates in fp32 TMEM (measured max ~2e-5 on these shapes).
+# CUDA-core path accumulates in fp32 (errors ~1e-7 to 6e-6); the tensor-core
+# path (g * q_len >= 8, bf16, D = 128) feeds each probability to the MMA as a
+# bf16 high part plus the remainder rounded to bf16 (relative error at most
+# 2^-15 per weight) and accumulates in fp32 TMEM: measured at most 1.45e-5
+# against the fp64 oracle on these shapes, so 5e-5 leaves a 3x margin.
 F32_ABS_CORE = 1e-5
-F32_ABS_TC = 1e-4
+F32_ABS_TC = 5e-5
 
 
 def f32_allowance(w):
@@ -281,3 +282,4 @@ def test_block_group_layouts_match_oracle(batch, len_range, paged):
     err = oracle.max_abs_diff(np64(out), ref)
     log_error(f"f32_out[groups_b{batch}_{'paged' if paged else 'contig'}]", err)
     assert err <= tol_for(w), f"max abs diff {err:.3e}"
+
