@@ -292,6 +292,7 @@ __global__ void __launch_bounds__(GROUPS == 2 ? 320 : (NTW == 1 ? 288 : 160))
     // ======================= producer warp ===============================
     int s = 0;
     bool failed = false;
+    const uint64_t pol = l2_evict_first();   // the cache is read once
     SegState p = st;
     for (; p.x < x1 && !failed; next_unit(a, p, seg_of(a, sPrefix, p, x1))) {
       const Seg sg = seg_of(a, sPrefix, p, x1);
@@ -335,8 +336,8 @@ __global__ void __launch_bounds__(GROUPS == 2 ? 320 : (NTW == 1 ? 288 : 160))
             mbar_arrive_expect_tx(&full[slot], 2 * bytes);
             if (bytes) {
               const size_t off = (((size_t)p.b * a.Hkv + p.hk) * a.max_seq_len + t0) * D;
-              bulk_g2s(dK, reinterpret_cast<const T*>(a.k_cache) + off, bytes, &full[slot]);
-              bulk_g2s(dV, reinterpret_cast<const T*>(a.v_cache) + off, bytes, &full[slot]);
+              bulk_g2s_hint(dK, reinterpret_cast<const T*>(a.k_cache) + off, bytes, &full[slot], pol);
+              bulk_g2s_hint(dV, reinterpret_cast<const T*>(a.v_cache) + off, bytes, &full[slot], pol);
             }
           }
         } else {
@@ -361,10 +362,10 @@ __global__ void __launch_bounds__(GROUPS == 2 ? 320 : (NTW == 1 ? 288 : 160))
           if (lane == 0) mbar_arrive_expect_tx(&full[slot], 2 * tot);
           __syncwarp();
           if (bytes) {
-            bulk_g2s(dK + (size_t)lane * kChunk * D, reinterpret_cast<const T*>(a.k_cache) + off,
-                     bytes, &full[slot]);
-            bulk_g2s(dV + (size_t)lane * kChunk * D, reinterpret_cast<const T*>(a.v_cache) + off,
-                     bytes, &full[slot]);
+            bulk_g2s_hint(dK + (size_t)lane * kChunk * D, reinterpret_cast<const T*>(a.k_cache) + off,
+                          bytes, &full[slot], pol);
+            bulk_g2s_hint(dV + (size_t)lane * kChunk * D, reinterpret_cast<const T*>(a.v_cache) + off,
+                          bytes, &full[slot], pol);
           }
         }
         __syncwarp();
@@ -653,8 +654,11 @@ __global__ void __launch_bounds__(GROUPS == 2 ? 320 : (NTW == 1 ? 288 : 160))
         else reinterpret_cast<float*>(a.out)[oi] = o;
         if (a.out_lse && d == 0) a.out_lse[row] = (L > 0.f) ? Ms + fast_log2(L) : -INFINITY;
       } else {
-        a.part_o[((size_t)slot_idx * a.R + rglob) * D + d] = o;
-        if (d == 0) a.part_lse[(size_t)slot_idx * a.R + rglob] = (L > 0.f) ? Ms + fast_log2(L) : -INFINITY;
+        // partials stay in L2 for the merge (evict_last)
+        const uint64_t keep = l2_evict_last();
+        st_hint(a.part_o + ((size_t)slot_idx * a.R + rglob) * D + d, o, keep);
+        if (d == 0)
+          st_hint(a.part_lse + (size_t)slot_idx * a.R + rglob, (L > 0.f) ? Ms + fast_log2(L) : -INFINITY, keep);
       }
     }
     named_bar_sync(bar, ncons);

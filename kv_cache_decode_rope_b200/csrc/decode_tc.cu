@@ -102,6 +102,7 @@ __device__ __forceinline__ void tc_loader(const DecodeArgs& a, const int* sPrefi
   int g = 0;
   bool failed = false;
   bool waited = false;   // programmatic-dependency wait done (before the first copy)
+  const uint64_t pol = l2_evict_first();   // the cache is read once
   // page id of chunk `ch` of sequence b (paged layout), -1 past `kend`
   auto page_of = [&](int b, int ch, int kend) -> int {
     if (ch >= kend) return -1;
@@ -156,8 +157,8 @@ __device__ __forceinline__ void tc_loader(const DecodeArgs& a, const int* sPrefi
       __syncwarp();
       if (row >= 0) {
         unsigned char* dst = ring + slot * (2 * DHALF) + lane * kChunk * 128;
-        tma_load_2d(dst, tm, 0, row, &fullb[slot]);
-        tma_load_2d(dst + DHALF, tm, 64, row, &fullb[slot]);
+        tma_load_2d_hint(dst, tm, 0, row, &fullb[slot], pol);
+        tma_load_2d_hint(dst + DHALF, tm, 64, row, &fullb[slot], pol);
       }
       __syncwarp();
     }
@@ -662,17 +663,18 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 for (int q4 = 0; q4 < NVAL / 4; ++q4)
                   dst[q4] = make_float4(ov[4 * q4], ov[4 * q4 + 1], ov[4 * q4 + 2], ov[4 * q4 + 3]);
               }
-            } else {
-              float4* dst = reinterpret_cast<float4*>(orow + dbase);
+            } else {   // partials stay in L2 for the merge (evict_last)
+              const uint64_t keep = l2_evict_last();
 #pragma unroll
               for (int q4 = 0; q4 < NVAL / 4; ++q4)
-                dst[q4] = make_float4(ov[4 * q4], ov[4 * q4 + 1], ov[4 * q4 + 2], ov[4 * q4 + 3]);
+                st_hint4(orow + dbase + 4 * q4, make_float4(ov[4 * q4], ov[4 * q4 + 1], ov[4 * q4 + 2], ov[4 * q4 + 3]),
+                         keep);
             }
           }
         }
         if (row_ok && hw == 0 && cs == 0) {
           const float lse = (L > 0.f) ? ms + fast_log2(L) : -INFINITY;
-          if (!whole) a.part_lse[(size_t)slot_idx * a.R + qr] = lse;
+          if (!whole) st_hint(a.part_lse + (size_t)slot_idx * a.R + qr, lse, l2_evict_last());
           else if (a.out_lse) a.out_lse[ob / TC_D] = lse;
         }
         tc_fence_before();  // the O reads above precede the next segment's first PV
