@@ -439,24 +439,47 @@ def measure(args, w, local, rank, world, steps, kernel_iters, e2e=False, cascade
     for _ in range(max(3, args.warmup)):
         e2e_step()
     torch.cuda.synchronize()
+    # the same calls and copies captured once as a CUDA graph, as a serving
+    # loop would replay them (--launch eager: plain calls)
+    run_e2e = e2e_step
+    if args.launch == "graph":
+        g_e2e = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(device=dev)
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            e2e_step()
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g_e2e):
+            e2e_step()
+        graphs.append(g_e2e)
+        run_e2e = g_e2e.replay
+        for _ in range(3):
+            run_e2e()
+        torch.cuda.synchronize()
     Ke = max(K, 20)
     if world > 1:
         torch.distributed.barrier()
-    e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(Ke)]
+    # Ke steps back to back between two events (flushed workloads: one by one)
+    e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(Ke if flush else 0)]
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record()
-    for a, b in e_ev:
+    for k in range(Ke):
         if flush:
             flush_buf.add_(1)
-        a.record()
-        e2e_step()
-        b.record()
+            e_ev[k][0].record()
+        run_e2e()
+        if flush:
+            e_ev[k][1].record()
     e1.record()
     torch.cuda.synchronize()
-    e2e_each = [a.elapsed_time(b) for a, b in e_ev]
-    res.update(e2e_ms=(sum(e2e_each) if flush else e0.elapsed_time(e1)) / Ke, e2e_each=e2e_each,
-               e2e_steps=Ke, h2d=h2d, d2h=d2h)
+    e2e_ms = (sum(a.elapsed_time(b) for a, b in e_ev) if flush else e0.elapsed_time(e1)) / Ke
+    e2e_each = timed(run_e2e, Ke)   # per-step distribution, after the timed region
+    res.update(e2e_ms=e2e_ms, e2e_each=e2e_each, e2e_steps=Ke, h2d=h2d, d2h=d2h,
+               e2e_launch="CUDA graph of the copies and the two library calls"
+               if args.launch == "graph" else "eager calls")
     del graphs
     return res
 
@@ -621,7 +644,7 @@ def main():
         "e2e": {"value": round(world * step_bytes / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
                 "us_per_step": round(e2e_ms * 1e3, 2),
                 "us_per_step_median": round(1e3 * statistics.median(r["e2e_each"]), 2),
-                "steps": r["e2e_steps"],
+                "steps": r["e2e_steps"], "launch": r["e2e_launch"],
                 "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
         "gpu_launches": (6 if args.cascade else 3) * K,
         "clocks": r["clocks"],
