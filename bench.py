@@ -413,25 +413,31 @@ def measure(args, w, local, rank, world, steps, kernel_iters, e2e=False, cascade
         del graphs
         return res
 
-    # ---- end to end: pinned host inputs -> device, step, output -> host
-    hq = q.cpu().pin_memory()
-    hk = kn.cpu().pin_memory()
-    hv = vn.cpu().pin_memory()
-    hs = seq.cpu().pin_memory()
-    hbt = bt.cpu().pin_memory() if bt is not None else None
+    # ---- end to end: the step's inputs (q, k_new, v_new, lengths, block
+    # table) staged in one pinned host buffer and copied to the device in one
+    # transfer, the step through the public API, the output copied back
+    segs = [q, kn, vn, seq] + ([bt] if bt is not None else [])
+    offs, tot = [], 0
+    for t in segs:
+        offs.append(tot)
+        tot += (t.numel() * t.element_size() + 255) // 256 * 256
+    hbuf = torch.empty(tot, dtype=torch.uint8).pin_memory()
+    dbuf = torch.empty(tot, dtype=torch.uint8, device=dev)
+
+    def view(buf, i):
+        t = segs[i]
+        return buf[offs[i]:offs[i] + t.numel() * t.element_size()].view(t.dtype).view(t.shape)
+
+    for i, t in enumerate(segs):
+        view(hbuf, i).copy_(t.cpu())
+    dq, dk, dv, ds = (view(dbuf, i) for i in range(4))
+    dbt = view(dbuf, 4) if bt is not None else None
     hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    dq, dk, dv, ds = (torch.empty_like(t) for t in (q, kn, vn, seq))
-    dbt = torch.empty_like(bt) if bt is not None else None
-    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hs) + ((hbt,) if hbt is not None else ()))
+    h2d = tot
     d2h = hout.numel() * hout.element_size()
 
     def e2e_step():
-        dq.copy_(hq, non_blocking=True)
-        dk.copy_(hk, non_blocking=True)
-        dv.copy_(hv, non_blocking=True)
-        ds.copy_(hs, non_blocking=True)
-        if dbt is not None:
-            dbt.copy_(hbt, non_blocking=True)
+        dbuf.copy_(hbuf, non_blocking=True)
         append(dq, dk, dv, ds, dbt, None)
         decode(dq, ds, dbt, None)
         hout.copy_(out, non_blocking=True)
