@@ -10,13 +10,15 @@
 // the 16-byte pieces of its q heads to rotate, of its k heads to rotate or
 // copy, and of its v heads to copy -- are cut into groups of 32, one per
 // warp.  A lane first asks for the sequence length (the only index read before
-// the programmatic-dependency wait), then, after the wait, issues the loads of
-// its q/k/v pieces at once, so both round trips overlap.  While those loads
-// are in flight the warp evaluates, in fp64, the r/2 rotation angles
-// pos * base^(-2j/r) (r = rotated width, D unless a partial rotary width is
-// asked for) and their sine and cosine (rope_sincos) into a table of its own
-// (a warp-level sync, no block barrier): positions reach 1e5+, where an fp32
-// angle would be off by ~1e-2 rad.  Each lane then rotates the pairs of its piece in fp64,
+// the programmatic-dependency wait) and evaluates the inverse frequencies
+// base^(-2j/r) of its pairs (r = rotated width, D unless a partial rotary
+// width is asked for) while it is in flight; after the wait it issues the
+// loads of its q/k/v pieces at once, so both round trips overlap.  While
+// those loads are in flight the warp evaluates, in fp64, the r/2 angles
+// pos * base^(-2j/r) and their sine and cosine (rope_sincos) into a table of
+// its own (a warp-level sync, no block barrier): positions reach 1e5+, where
+// an fp32 angle would be off by ~1e-2 rad.  Each lane then rotates the pairs
+// of its piece in fp64,
 // rounding once to the storage type: EPV half-split pairs (j, j + r/2) from
 // two pieces, or EPV/2 interleaved pairs (2j, 2j + 1) from one.  Pieces past r
 // are copied unrotated (k), or left in place (q), and v is copied.  q is
@@ -121,18 +123,16 @@ __global__ void __launch_bounds__(kAppendWarps * 32) append_rope_kernel(AppendAr
   // loads below are pending
   const int Lraw = a.seq_lens[b];
   const int sstart = a.shard_start ? a.shard_start[b] : 0;
-  // inverse frequencies of the lane's pairs j = lane + 32 m (independent of
-  // the position, so they are ready when the length arrives):
-  // base^(-2j/r) = 2^(-2j/r log2 base)
+  // inverse frequencies base^(-2j/r) of the lane's pairs j = lane + 32 m,
+  // independent of the position: evaluated while the length load is in
+  // flight (pow, accurate to the last bits: at positions near 2^30 an error
+  // of 1e-15 in the frequency would move the angle by 1e-6 rad)
   constexpr int NPL = (HALF + 31) / 32;        // pairs per lane (at most)
   const int RH = a.rot / 2;                     // rotated pairs per head row
   double inv_freq[NPL];
-  {
-    const double lb = log2(a.rope_base);
 #pragma unroll
-    for (int m = 0; m < NPL; ++m)
-      inv_freq[m] = exp2(-2.0 * (double)(lane + 32 * m) / (double)a.rot * lb);
-  }
+  for (int m = 0; m < NPL; ++m)
+    inv_freq[m] = pow(a.rope_base, -2.0 * (double)(lane + 32 * m) / (double)a.rot);
   // everything else (q, k/v, the caches, the status word) only after the
   // previous kernel has finished
   grid_dep_wait();
