@@ -1,8 +1,10 @@
 """Benchmark of one KV-cache decode step: RoPE + KV append + GQA flash decode.
 
-A step is one pass of the whole path over one batch: ``kv_append_rope``
-(rotate the new tokens, append k/v) followed by ``decode_attention[_paged]``
-(split-KV attention + log-sum-exp merge).  Inputs are resident in HBM before
+A step is one pass of the whole path over one batch: one ``kvd_decode_step``
+call, which rotates the new tokens and appends k/v (the ``kv_append_rope``
+kernel), then runs split-KV attention and the log-sum-exp merge (the
+``decode_attention[_paged]`` kernels); ``--step-route two-calls`` makes the
+same step from the two separate calls.  Inputs are resident in HBM before
 the timed region; the KV cache is larger than the 126 MB L2 for every default
 workload, so no flush is needed between steps (the tiny workload is flushed).
 ``value`` is algorithmic bytes per step (see workloads.step_bytes) divided by
@@ -69,6 +71,9 @@ def parse():
                          "workload's geometry: one token per step, graph replay vs eager calls")
     ap.add_argument("--launch", default="graph", choices=["graph", "eager"],
                     help="replay the step's library calls from CUDA graphs (default) or call them eagerly")
+    ap.add_argument("--step-route", default="one-call", choices=["one-call", "two-calls"],
+                    help="a step as one kvd_decode_step call (default) or as kv_append_rope then "
+                         "decode_attention[_paged]")
     return ap.parse_args()
 
 
@@ -307,13 +312,25 @@ def measure(args, w, local, rank, world, steps, kernel_iters, e2e=False, cascade
             kvd.decode_attention_paged(q, inp["k_cache"], inp["v_cache"], seq, bt_, out, scale=w.scale,
                                        max_kv_len=mkl, workspace=ws, status=st)
 
+    one_call = args.step_route == "one-call" and not cascade
+
+    def step_calls(q, kn, vn, seq, bt_=bt, st=status):
+        """One step through the public API: kvd_decode_step (one library
+        call; on the CUDA-core path the decode kernel appends the new tokens
+        itself), or kv_append_rope then decode_attention[_paged]."""
+        if one_call:
+            kvd.decode_step(q, kn, vn, inp["k_cache"], inp["v_cache"], seq, bt_, out, scale=w.scale,
+                            max_kv_len=mkl, workspace=ws, rope_base=w.rope_base, status=st)
+        else:
+            append(q, kn, vn, seq, bt_, st)
+            decode(q, seq, bt_, st)
+
     q, kn, vn, seq = inp["q"], inp["k_new"], inp["v_new"], inp["seq_lens"]
     for _ in range(args.warmup):
-        append(q, kn, vn, seq)
-        decode(q, seq)
+        step_calls(q, kn, vn, seq)
     torch.cuda.synchronize()
 
-    # The timed loop replays the step's two library calls from a CUDA graph
+    # The timed loop replays the step's library call(s) from a CUDA graph
     # captured through the same public API: the kernels, their arguments and
     # the work are those of the eager calls, but the host enqueues a step in a
     # few microseconds, so the device never idles waiting for Python, and the
@@ -326,14 +343,14 @@ def measure(args, w, local, rank, world, steps, kernel_iters, e2e=False, cascade
         side = torch.cuda.Stream(device=dev)
         side.wait_stream(torch.cuda.current_stream())
         with torch.cuda.stream(side):
+            step_calls(q, kn, vn, seq)
             append(q, kn, vn, seq)
             decode(q, seq)
         torch.cuda.current_stream().wait_stream(side)
         torch.cuda.synchronize()
         g_step, g_app, g_dec = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
         with torch.cuda.graph(g_step):
-            append(q, kn, vn, seq)
-            decode(q, seq)
+            step_calls(q, kn, vn, seq)
         with torch.cuda.graph(g_app):
             append(q, kn, vn, seq)
         with torch.cuda.graph(g_dec):
@@ -354,8 +371,7 @@ def measure(args, w, local, rank, world, steps, kernel_iters, e2e=False, cascade
             decode(q, seq)
 
         def run_step():
-            run_append()
-            run_decode()
+            step_calls(q, kn, vn, seq)
 
     def timed(fn, n, before=None):
         """Per-iteration device times (ms) of n calls of fn, each after an
@@ -407,7 +423,7 @@ def measure(args, w, local, rank, world, steps, kernel_iters, e2e=False, cascade
     if status.item() != 0:
         raise RuntimeError(f"device status flags set during the bench of {w.name}: {status.item()}")
 
-    res = dict(total_ms=total_ms, steps=K, step_ms=step_ms, dec_ms=dec_ms, app_ms=app_ms, bytes=nbytes,
+    res = dict(one_call=one_call, total_ms=total_ms, steps=K, step_ms=step_ms, dec_ms=dec_ms, app_ms=app_ms, bytes=nbytes,
                clocks=clk.summary(), flush=flush, cache_bytes=cache_bytes, w=w, mkl=mkl)
     if not e2e:
         del graphs
@@ -438,8 +454,7 @@ def measure(args, w, local, rank, world, steps, kernel_iters, e2e=False, cascade
 
     def e2e_step():
         dbuf.copy_(hbuf, non_blocking=True)
-        append(dq, dk, dv, ds, dbt, None)
-        decode(dq, ds, dbt, None)
+        step_calls(dq, dk, dv, ds, dbt, None)
         hout.copy_(out, non_blocking=True)
 
     for _ in range(max(3, args.warmup)):
@@ -484,7 +499,7 @@ def measure(args, w, local, rank, world, steps, kernel_iters, e2e=False, cascade
     e2e_ms = (sum(a.elapsed_time(b) for a, b in e_ev) if flush else e0.elapsed_time(e1)) / Ke
     e2e_each = timed(run_e2e, Ke)   # per-step distribution, after the timed region
     res.update(e2e_ms=e2e_ms, e2e_each=e2e_each, e2e_steps=Ke, h2d=h2d, d2h=d2h,
-               e2e_launch="CUDA graph of the copies and the two library calls"
+               e2e_launch="CUDA graph of the copies and the step's library call(s)"
                if args.launch == "graph" else "eager calls")
     del graphs
     return res
@@ -623,10 +638,12 @@ def main():
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
             "l2": ("flushed between steps" if r["flush"] else
                    f"inputs larger than L2 ({r['cache_bytes'] / 2**20:.0f} MiB KV cache)"),
-            "step": "kv_append_rope + " + ("cascade decode (prefix per group + suffix + merge)"
-                                           if args.cascade else
-                                           "decode_attention" + ("_paged" if w.paged else "")),
-            "launch": "CUDA graph replay of the two library calls" if args.launch == "graph" else "eager calls",
+            "step": ("kv_append_rope + cascade decode (prefix per group + suffix + merge)" if args.cascade
+                     else "kvd_decode_step (kv_append_rope + decode_attention" + ("_paged" if w.paged else "")
+                     + " in one call)" if r["one_call"] else
+                     "kv_append_rope + decode_attention" + ("_paged" if w.paged else "")),
+            "launch": "CUDA graph replay of the step's library call(s)" if args.launch == "graph"
+                      else "eager calls",
             "max_kv_len": r["mkl"]}),
         "step_us": dist_us(r["step_ms"]),
         "roofline": {
